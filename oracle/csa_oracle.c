@@ -1,0 +1,487 @@
+/*
+ * csa_oracle.c -- plain, slow, fp64 CPU oracle for the Compressed Sparse
+ * Attention (CSA) / Heavily Compressed Attention (HCA) hot path.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing on the product path may call, link or
+ * load this file: only the test suite, the smoke check and the CPU-baseline
+ * leg of the benchmark use it.  It shares no code, header, table or helper
+ * with the CUDA library.
+ *
+ * Every function computes its definition literally: nested loops, fp64
+ * accumulation, exp() in double, inputs decoded from the exact bf16 / fp32
+ * bits the GPU receives.  Sources (all prose; the pages never write the
+ * equations out, so the formulas below are the plain readings stated at each
+ * function):
+ *   [A4] "Anatomy of a Frontier Model: Reading DeepSeek-V4 Through Part V",
+ *        section "The attention: compress, then select" (CSA and HCA bullets)
+ *        and its "three details" (sliding window, sink, QK-norm/RoPE);
+ *        section "The skeleton, and what's kept" (single shared KV head,
+ *        entry is both key and value).
+ *   [E1] "The Exchange Rates of a Million Tokens", section 3 "Rate #2: bytes
+ *        buy budget, and spend recall" (two overlapping series under one
+ *        joint softmax; ReLU-gated indexer; top-k).
+ *   [N3] "DeepSeek V4: How It Made Million-Token AI", section "The Memory
+ *        Problem Nobody Wanted to Solve" (learned, not average, pooling;
+ *        HCA every 128 tokens; 128-token window).
+ *
+ * Parallelism: OpenMP over independent outputs only.  Each output element is
+ * computed by one thread with a fixed loop order, so results do not depend on
+ * the thread count.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+enum { ORC_F32 = 0, ORC_BF16 = 1 };
+enum {
+  ORC_OK = 0,
+  ORC_ERR_ARG = -1,     /* bad sizes / dtype / null pointer            */
+  ORC_ERR_POS = -2,     /* a query position outside its sequence       */
+  ORC_ERR_NAN = -3,     /* a NaN score reached the selector            */
+  ORC_ERR_CACHE = -4    /* visible entries exceed the cache rows        */
+};
+
+/* ------------------------------------------------------------------ */
+/* number formats                                                      */
+/* ------------------------------------------------------------------ */
+
+/* Decode element i of a buffer holding fp32 or bf16 (upper 16 bits of an
+ * IEEE-754 binary32) values.  Both conversions to double are exact. */
+static double ld(const void *p, int dt, size_t i) {
+  if (dt == ORC_F32) return (double)((const float *)p)[i];
+  uint32_t u = ((uint32_t)((const uint16_t *)p)[i]) << 16;
+  float f;
+  memcpy(&f, &u, 4);
+  return (double)f;
+}
+
+/* Round a double to the nearest bf16 value, ties to even, directly from the
+ * real value (no intermediate fp32 rounding).  bf16 keeps 8 significant bits
+ * and the binary32 exponent range; below 2^-126 the spacing is 2^-133. */
+static uint16_t bf16_from_double(double v) {
+  if (isnan(v)) return (uint16_t)0x7FC0;
+  if (isinf(v)) return v > 0 ? (uint16_t)0x7F80 : (uint16_t)0xFF80;
+  if (v == 0.0) return signbit(v) ? (uint16_t)0x8000 : (uint16_t)0x0000;
+  double a = fabs(v), r;
+  int e;
+  (void)frexp(a, &e);                   /* a = f * 2^e, 0.5 <= f < 1 */
+  int q = e - 8;                        /* weight of the last kept bit */
+  if (q < -133) q = -133;               /* subnormal range */
+  r = nearbyint(ldexp(a, -q));          /* default rounding: ties to even */
+  r = ldexp(r, q);
+  float f = (float)r;                   /* exact: r is a bf16 value (or inf) */
+  if (r >= 0x1p128) f = INFINITY;
+  uint32_t u;
+  memcpy(&u, &f, 4);
+  uint16_t h = (uint16_t)(u >> 16);
+  return v < 0 ? (uint16_t)(h | 0x8000) : h;
+}
+
+/* Round n doubles to the output dtype (fp32: C's round-to-nearest-even
+ * conversion; bf16: bf16_from_double). */
+int orc_round(const double *in, size_t n, int dt, void *out) {
+  if (!in || !out) return ORC_ERR_ARG;
+  if (dt == ORC_F32) {
+    for (size_t i = 0; i < n; ++i) ((float *)out)[i] = (float)in[i];
+  } else if (dt == ORC_BF16) {
+    for (size_t i = 0; i < n; ++i) ((uint16_t *)out)[i] = bf16_from_double(in[i]);
+  } else {
+    return ORC_ERR_ARG;
+  }
+  return ORC_OK;
+}
+
+void orc_set_threads(int n) {
+#ifdef _OPENMP
+  if (n > 0) omp_set_num_threads(n);
+#else
+  (void)n;
+#endif
+}
+
+int orc_get_threads(void) {
+#ifdef _OPENMP
+  return omp_get_max_threads();
+#else
+  return 1;
+#endif
+}
+
+static long ceil_div(long a, long b) { return (a + b - 1) / b; }
+
+/* ------------------------------------------------------------------ */
+/* a1: CSA overlapping compressor                                      */
+/* ------------------------------------------------------------------ */
+/*
+ * [A4] CSA bullet: every 4 tokens become one entry, a learned softmax-
+ * weighted pooling of their key-value vectors, per channel, with learned
+ * position biases; each entry pools 8 tokens, its own block and the one
+ * before.  [E1] section 3: two series C^a / C^b over the overlapping blocks,
+ * one joint softmax.  [N3]: learned weights, not average pooling.
+ *
+ * Reading (the pages do not print the formula):
+ *   entry i of sequence b pools slots j = 0..7, token s = 4(i-1) + j;
+ *   slots 0..3 (block i-1) use series a, slots 4..7 (block i) series b:
+ *     z_s[c] = sum_e x_s[e] * W[e][c] + beta[j][c],  W = Wa (j<4) or Wb,
+ *   tokens outside [0, n_b) are masked (no term in the softmax), so entry 0
+ *   pools only its own 4 tokens and a trailing partial block pools what
+ *   exists; per channel c:
+ *     C_i[c] = sum_s softmax_s(z_s[c]) * x_s[c].
+ * Output rows i >= ceil(n_b/4) are zero.  out: [B][ceil(n_max/4)][d].
+ */
+int orc_csa_compress(const void *x, const int32_t *lens, int B, int n_max, int d,
+                     const void *Wa, const void *Wb, const void *beta, int dt,
+                     double *out) {
+  if (!x || !lens || !Wa || !Wb || !beta || !out) return ORC_ERR_ARG;
+  if (B < 0 || n_max < 0 || d <= 0 || (dt != ORC_F32 && dt != ORC_BF16)) return ORC_ERR_ARG;
+  const long nc_max = ceil_div(n_max, 4);
+  for (int b = 0; b < B; ++b)
+    if (lens[b] < 0 || lens[b] > n_max) return ORC_ERR_ARG;
+  long total = (long)B * nc_max;
+  int err = ORC_OK;
+#pragma omp parallel for schedule(dynamic, 4)
+  for (long bi = 0; bi < total; ++bi) {
+    const int b = (int)(bi / nc_max);
+    const long i = bi % nc_max;
+    const long nb = lens[b];
+    double *o = out + (size_t)bi * d;
+    if (i >= ceil_div(nb, 4)) {
+      for (int c = 0; c < d; ++c) o[c] = 0.0;
+      continue;
+    }
+    double *z = (double *)malloc(sizeof(double) * 8 * (size_t)d);
+    int valid[8];
+    if (!z) { err = ORC_ERR_ARG; continue; }
+    for (int j = 0; j < 8; ++j) {
+      const long s = 4 * (i - 1) + j;
+      valid[j] = (s >= 0 && s < nb);
+      if (!valid[j]) continue;
+      const void *W = (j < 4) ? Wa : Wb;
+      const size_t xrow = ((size_t)b * n_max + (size_t)s) * d;
+      for (int c = 0; c < d; ++c) {
+        double acc = 0.0;
+        for (int e = 0; e < d; ++e) acc += ld(x, dt, xrow + e) * ld(W, dt, (size_t)e * d + c);
+        z[j * d + c] = acc + ld(beta, dt, (size_t)j * d + c);
+      }
+    }
+    for (int c = 0; c < d; ++c) {
+      double mx = -INFINITY;
+      for (int j = 0; j < 8; ++j)
+        if (valid[j] && z[j * d + c] > mx) mx = z[j * d + c];
+      double den = 0.0, num = 0.0;
+      for (int j = 0; j < 8; ++j) {
+        if (!valid[j]) continue;
+        const long s = 4 * (i - 1) + j;
+        const double p = exp(z[j * d + c] - mx);
+        den += p;
+        num += p * ld(x, dt, ((size_t)b * n_max + (size_t)s) * d + c);
+      }
+      o[c] = num / den;
+    }
+    free(z);
+  }
+  return err;
+}
+
+/* ------------------------------------------------------------------ */
+/* a2: HCA compressor                                                  */
+/* ------------------------------------------------------------------ */
+/*
+ * [A4] HCA bullet: every m = 128 tokens become one entry, without overlap.
+ * [N3]: every 128 tokens collapse into a single KV entry.  Reading: the same
+ * softmax-weighted per-channel pooling as CSA with a single series:
+ *   z_s[c] = sum_e x_s[e] * W[e][c] + beta[s - m*i][c],  s in block i,
+ *   C_i[c] = sum_s softmax_s(z_s[c]) * x_s[c]  (valid s < n_b only).
+ * Output rows i >= ceil(n_b/m) are zero.  out: [B][ceil(n_max/m)][d].
+ */
+int orc_hca_compress(const void *x, const int32_t *lens, int B, int n_max, int d, int m,
+                     const void *W, const void *beta, int dt, double *out) {
+  if (!x || !lens || !W || !beta || !out) return ORC_ERR_ARG;
+  if (B < 0 || n_max < 0 || d <= 0 || m <= 0 || (dt != ORC_F32 && dt != ORC_BF16)) return ORC_ERR_ARG;
+  const long nc_max = ceil_div(n_max, m);
+  for (int b = 0; b < B; ++b)
+    if (lens[b] < 0 || lens[b] > n_max) return ORC_ERR_ARG;
+  long total = (long)B * nc_max;
+  int err = ORC_OK;
+#pragma omp parallel for schedule(dynamic, 1)
+  for (long bi = 0; bi < total; ++bi) {
+    const int b = (int)(bi / nc_max);
+    const long i = bi % nc_max;
+    const long nb = lens[b];
+    double *o = out + (size_t)bi * d;
+    if (i >= ceil_div(nb, m)) {
+      for (int c = 0; c < d; ++c) o[c] = 0.0;
+      continue;
+    }
+    long cnt = nb - (long)m * i;
+    if (cnt > m) cnt = m;
+    double *z = (double *)malloc(sizeof(double) * (size_t)cnt * d);
+    if (!z) { err = ORC_ERR_ARG; continue; }
+    for (long j = 0; j < cnt; ++j) {
+      const size_t xrow = ((size_t)b * n_max + (size_t)(m * i + j)) * d;
+      for (int c = 0; c < d; ++c) {
+        double acc = 0.0;
+        for (int e = 0; e < d; ++e) acc += ld(x, dt, xrow + e) * ld(W, dt, (size_t)e * d + c);
+        z[j * d + c] = acc + ld(beta, dt, (size_t)j * d + c);
+      }
+    }
+    for (int c = 0; c < d; ++c) {
+      double mx = -INFINITY;
+      for (long j = 0; j < cnt; ++j)
+        if (z[j * d + c] > mx) mx = z[j * d + c];
+      double den = 0.0, num = 0.0;
+      for (long j = 0; j < cnt; ++j) {
+        const double p = exp(z[j * d + c] - mx);
+        den += p;
+        num += p * ld(x, dt, ((size_t)b * n_max + (size_t)(m * i + j)) * d + c);
+      }
+      o[c] = num / den;
+    }
+    free(z);
+  }
+  return err;
+}
+
+/* ------------------------------------------------------------------ */
+/* query positions and visibility                                      */
+/* ------------------------------------------------------------------ */
+/*
+ * [A4] "three details": a compressed entry exists only once its block is
+ * complete, so a query at 0-based position t sees entries i < floor((t+1)/m).
+ * Position of query (b, tq): q_pos[b][tq] if given, else lens[b] - Tq + tq
+ * (the last Tq tokens of the sequence; t = n - 1 for a decode step).
+ */
+static int query_pos(const int32_t *lens, const int32_t *q_pos, int b, int Tq, int tq, long *t) {
+  long v = q_pos ? (long)q_pos[(size_t)b * Tq + tq] : (long)lens[b] - Tq + tq;
+  if (v < 0 || v >= lens[b]) return ORC_ERR_POS;
+  *t = v;
+  return ORC_OK;
+}
+
+/* ------------------------------------------------------------------ */
+/* a3: lightning indexer scores                                        */
+/* ------------------------------------------------------------------ */
+/*
+ * [A4] CSA bullet: a small "lightning indexer", 64 heads of 128 dimensions,
+ * ranks the compressed blocks for each query.  [E1] section 3: ReLU-gated
+ * dot products.  Reading (no scale; a positive global scale does not change
+ * the ranking):
+ *   I[t,i] = sum_h w[t,h] * max(0, sum_e qI[t,h,e] * kI[i,e]),
+ *   for visible i < floor((t+1)/4); invisible entries get -inf.
+ * qI: [B][Tq][HI][dI], w: [B][Tq][HI], kI: [B][nc_max][dI],
+ * scores: [B][Tq][nc_max] (double).
+ */
+int orc_index_scores(const void *qI, const void *w, const void *kI, const int32_t *lens,
+                     const int32_t *q_pos, int B, int Tq, int HI, int dI, int nc_max,
+                     int dt, double *scores) {
+  if (!qI || !w || !kI || !lens || !scores) return ORC_ERR_ARG;
+  if (B < 0 || Tq < 0 || HI <= 0 || dI <= 0 || nc_max < 0) return ORC_ERR_ARG;
+  if (dt != ORC_F32 && dt != ORC_BF16) return ORC_ERR_ARG;
+  int err = ORC_OK;
+  const long R = (long)B * Tq;
+  long *vis = (long *)malloc(sizeof(long) * (size_t)(R > 0 ? R : 1));
+  if (!vis) return ORC_ERR_ARG;
+  for (long r = 0; r < R; ++r) {
+    long t;
+    vis[r] = 0;
+    if (query_pos(lens, q_pos, (int)(r / Tq), Tq, (int)(r % Tq), &t) != ORC_OK) {
+      err = ORC_ERR_POS;
+      continue;
+    }
+    vis[r] = (t + 1) / 4;
+    if (vis[r] > nc_max) { err = ORC_ERR_CACHE; vis[r] = 0; }
+  }
+  /* every score is independent: parallel over (query row, entry) */
+  const long total = R * (long)nc_max;
+#pragma omp parallel for schedule(static)
+  for (long ri = 0; ri < total; ++ri) {
+    const long r = ri / nc_max, i = ri % nc_max;
+    const int b = (int)(r / Tq);
+    if (i >= vis[r]) { scores[ri] = -INFINITY; continue; }
+    double acc = 0.0;
+    for (int h = 0; h < HI; ++h) {
+      double dot = 0.0;
+      const size_t qrow = ((size_t)r * HI + h) * dI;
+      const size_t krow = ((size_t)b * nc_max + i) * dI;
+      for (int e = 0; e < dI; ++e) dot += ld(qI, dt, qrow + e) * ld(kI, dt, krow + e);
+      acc += ld(w, dt, (size_t)r * HI + h) * (dot > 0.0 ? dot : 0.0);
+    }
+    scores[ri] = acc;
+  }
+  free(vis);
+  return err;
+}
+
+/* ------------------------------------------------------------------ */
+/* a4: per-query top-k                                                 */
+/* ------------------------------------------------------------------ */
+/*
+ * [A4] CSA bullet: each query attends to only the 1,024 (Flash: 512) most
+ * relevant entries chosen by the indexer.  Reading: the selected set is the
+ * k visible entries that come first in the total order (score descending,
+ * index ascending) -- ties go to the lower index, and -0.0 ranks as +0.0
+ * (the double comparisons below treat them as equal); every visible entry
+ * if fewer than k are visible.  Output: the set in ascending index order,
+ * padded with -1.  scores: [R][nc_max], vis: [R], idx: [R][k].
+ */
+typedef struct { double s; int32_t i; } orc_item;
+
+static int cmp_rank(const void *pa, const void *pb) {
+  const orc_item *a = (const orc_item *)pa, *b = (const orc_item *)pb;
+  if (a->s > b->s) return -1;
+  if (a->s < b->s) return 1;
+  return (a->i < b->i) ? -1 : (a->i > b->i);
+}
+
+static int cmp_i32(const void *pa, const void *pb) {
+  int32_t a = *(const int32_t *)pa, b = *(const int32_t *)pb;
+  return (a > b) - (a < b);
+}
+
+int orc_select_topk(const double *scores, const int32_t *vis, long R, int nc_max, int k,
+                    int32_t *idx) {
+  if (!scores || !vis || !idx || R < 0 || nc_max < 0 || k <= 0) return ORC_ERR_ARG;
+  int err = ORC_OK;
+#pragma omp parallel for schedule(dynamic, 1)
+  for (long r = 0; r < R; ++r) {
+    long v = vis[r];
+    int32_t *orow = idx + (size_t)r * k;
+    for (int j = 0; j < k; ++j) orow[j] = -1;
+    if (v < 0 || v > nc_max) { err = ORC_ERR_ARG; continue; }
+    orc_item *items = (orc_item *)malloc(sizeof(orc_item) * (size_t)(v > 0 ? v : 1));
+    if (!items) { err = ORC_ERR_ARG; continue; }
+    int bad = 0;
+    for (long i = 0; i < v; ++i) {
+      items[i].s = scores[(size_t)r * nc_max + i];
+      items[i].i = (int32_t)i;
+      if (isnan(items[i].s)) bad = 1;
+    }
+    if (bad) { err = ORC_ERR_NAN; free(items); continue; }
+    qsort(items, (size_t)v, sizeof(orc_item), cmp_rank);
+    long take = v < k ? v : k;
+    for (long j = 0; j < take; ++j) orow[j] = items[j].i;
+    qsort(orow, (size_t)take, sizeof(int32_t), cmp_i32);
+    free(items);
+  }
+  return err;
+}
+
+/* Visible-entry counts floor((t+1)/m) per query row, for the selector. */
+int orc_visible(const int32_t *lens, const int32_t *q_pos, int B, int Tq, int m, int32_t *vis) {
+  if (!lens || !vis || B < 0 || Tq < 0 || m <= 0) return ORC_ERR_ARG;
+  int err = ORC_OK;
+  for (int b = 0; b < B; ++b)
+    for (int tq = 0; tq < Tq; ++tq) {
+      long t;
+      if (query_pos(lens, q_pos, b, Tq, tq, &t) != ORC_OK) {
+        err = ORC_ERR_POS;
+        vis[(size_t)b * Tq + tq] = 0;
+        continue;
+      }
+      vis[(size_t)b * Tq + tq] = (int32_t)((t + 1) / m);
+    }
+  return err;
+}
+
+/* ------------------------------------------------------------------ */
+/* a5 / a6: attention over selected (CSA) or all (HCA) entries + window */
+/* ------------------------------------------------------------------ */
+/*
+ * [A4] "The skeleton": one key-value head shared by every query head; each
+ * cached entry is both the key and the value.  CSA bullet: each query
+ * attends to its selected entries.  HCA bullet: queries attend to all
+ * entries densely.  "Three details": every CSA and HCA layer also attends to
+ * the last 128 tokens directly.  Reading: for each head h,
+ *   keys = {C_i : i in S_t} + {x_s : max(0, t-W+1) <= s <= t}, one joint
+ *   softmax (no de-duplication), logits l = scale * (q[t,h] . v),
+ *   o[t,h] = sum softmax(l) * v.
+ * S_t: the entries of idx[b][tq][:] with 0 <= i < floor((t+1)/m) (others,
+ * including the -1 padding, contribute nothing); idx == NULL selects every
+ * visible entry (HCA).  The window token at position s is row (s mod n_tok)
+ * of kv_tok[b] (a ring: it must hold the query's whole window,
+ * min(W, t+1) <= n_tok).  scale <= 0 means 1/sqrt(d).
+ * q: [B][Tq][H][d], kv_c: [B][nc_max][d], kv_tok: [B][n_tok][d],
+ * idx: [B][Tq][k], out: [B][Tq][H][d] (double).
+ */
+int orc_attend(const void *q, const void *kv_c, const void *kv_tok, int n_tok,
+               const int32_t *idx, const int32_t *lens, const int32_t *q_pos, int B, int Tq,
+               int H, int d, int nc_max, int k, int window, int m, double scale, int dt,
+               double *out) {
+  if (!q || !kv_tok || !lens || !out) return ORC_ERR_ARG;
+  if (B < 0 || Tq < 0 || H <= 0 || d <= 0 || nc_max < 0 || window <= 0 || m <= 0) return ORC_ERR_ARG;
+  if (n_tok <= 0 || (idx && k <= 0) || (nc_max > 0 && !kv_c)) return ORC_ERR_ARG;
+  if (dt != ORC_F32 && dt != ORC_BF16) return ORC_ERR_ARG;
+  if (!(scale > 0.0)) scale = 1.0 / sqrt((double)d);
+  int err = ORC_OK;
+  const long R = (long)B * Tq;
+#pragma omp parallel for schedule(dynamic, 1)
+  for (long r = 0; r < R; ++r) {
+    const int b = (int)(r / Tq), tq = (int)(r % Tq);
+    double *orow = out + (size_t)r * H * d;
+    long t;
+    if (query_pos(lens, q_pos, b, Tq, tq, &t) != ORC_OK) {
+      err = ORC_ERR_POS;
+      for (long j = 0; j < (long)H * d; ++j) orow[j] = 0.0;
+      continue;
+    }
+    long vis = (t + 1) / m;
+    if (vis > nc_max) {
+      err = ORC_ERR_CACHE;
+      for (long j = 0; j < (long)H * d; ++j) orow[j] = 0.0;
+      continue;
+    }
+    /* the key list: selected entries (as cache rows), then window tokens */
+    long nsel = idx ? k : vis;
+    long w0 = t - window + 1;
+    if (w0 < 0) w0 = 0;
+    long nwin = t - w0 + 1;
+    if (nwin > n_tok) {   /* the ring cannot hold this query's window */
+      err = ORC_ERR_ARG;
+      for (long j = 0; j < (long)H * d; ++j) orow[j] = 0.0;
+      continue;
+    }
+    double *keys = (double *)malloc(sizeof(double) * (size_t)(nsel + nwin) * d);
+    if (!keys) { err = ORC_ERR_ARG; continue; }
+    long nk = 0;
+    for (long j = 0; j < nsel; ++j) {
+      long i = idx ? (long)idx[(size_t)r * k + j] : j;
+      if (i < 0 || i >= vis) continue;
+      for (int e = 0; e < d; ++e) keys[nk * d + e] = ld(kv_c, dt, ((size_t)b * nc_max + i) * d + e);
+      ++nk;
+    }
+    for (long s = w0; s <= t; ++s) {
+      const size_t row = (size_t)b * n_tok + (size_t)(s % n_tok);
+      for (int e = 0; e < d; ++e) keys[nk * d + e] = ld(kv_tok, dt, row * d + e);
+      ++nk;
+    }
+    double *lg = (double *)malloc(sizeof(double) * (size_t)nk);
+    if (!lg) { free(keys); err = ORC_ERR_ARG; continue; }
+    for (int h = 0; h < H; ++h) {
+      const size_t qrow = ((size_t)r * H + h) * d;
+      double mx = -INFINITY;
+      for (long j = 0; j < nk; ++j) {
+        double dot = 0.0;
+        for (int e = 0; e < d; ++e) dot += ld(q, dt, qrow + e) * keys[j * d + e];
+        lg[j] = scale * dot;
+        if (lg[j] > mx) mx = lg[j];
+      }
+      double den = 0.0;
+      for (long j = 0; j < nk; ++j) {
+        lg[j] = exp(lg[j] - mx);
+        den += lg[j];
+      }
+      for (int e = 0; e < d; ++e) {
+        double acc = 0.0;
+        for (long j = 0; j < nk; ++j) acc += lg[j] * keys[j * d + e];
+        orow[(size_t)h * d + e] = acc / den;
+      }
+    }
+    free(lg);
+    free(keys);
+  }
+  return err;
+}

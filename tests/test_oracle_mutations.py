@@ -1,0 +1,69 @@
+"""Mutation check of the oracle's pins: each plausible mistake below (a
+swapped series, a transposed weight, a dropped ReLU or head weight, an
+off-by-one in visibility or the window, a wrong tie rule, a wrong scale,
+double rounding) is planted in a copy of the oracle's C source, compiled,
+and the pin tests are run against it.  Every mutant must fail at least one
+pin; a mutant that survives means the pins do not determine that part of
+the definition."""
+import os
+import subprocess
+import sys
+import tempfile
+from concurrent.futures import ThreadPoolExecutor
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+SRC = os.path.join(ROOT, "oracle", "csa_oracle.c")
+PINS = ["tests/test_oracle_compress.py", "tests/test_oracle_index_topk.py",
+        "tests/test_oracle_attend.py", "tests/test_oracle_e2e.py"]
+
+MUTANTS = {
+    "csa_series_swapped": ("const void *W = (j < 4) ? Wa : Wb;", "const void *W = (j < 4) ? Wb : Wa;"),
+    "csa_slot_order_reversed": ("z[j * d + c] = acc + ld(beta, dt, (size_t)j * d + c);\n      }\n    }\n    for (int c = 0; c < d; ++c) {\n      double mx = -INFINITY;\n      for (int j = 0; j < 8; ++j)",
+                                "z[j * d + c] = acc + ld(beta, dt, (size_t)(7 - j) * d + c);\n      }\n    }\n    for (int c = 0; c < d; ++c) {\n      double mx = -INFINITY;\n      for (int j = 0; j < 8; ++j)"),
+    "csa_no_overlap": ("const long s = 4 * (i - 1) + j;\n      valid[j] = (s >= 0 && s < nb);",
+                       "const long s = 4 * (i - 1) + j;\n      valid[j] = (s >= 4 * i && s < nb);"),
+    "weight_transposed": ("acc += ld(x, dt, xrow + e) * ld(W, dt, (size_t)e * d + c);\n        z[j * d + c] = acc + ld(beta, dt, (size_t)j * d + c);\n      }\n    }\n    for (int c = 0; c < d; ++c) {\n      double mx = -INFINITY;\n      for (int j = 0; j < 8; ++j)",
+                          "acc += ld(x, dt, xrow + e) * ld(W, dt, (size_t)c * d + e);\n        z[j * d + c] = acc + ld(beta, dt, (size_t)j * d + c);\n      }\n    }\n    for (int c = 0; c < d; ++c) {\n      double mx = -INFINITY;\n      for (int j = 0; j < 8; ++j)"),
+    "hca_bias_ignored": ("z[j * d + c] = acc + ld(beta, dt, (size_t)j * d + c);\n      }\n    }\n    for (int c = 0; c < d; ++c) {\n      double mx = -INFINITY;\n      for (long j = 0;",
+                         "z[j * d + c] = acc;\n      }\n    }\n    for (int c = 0; c < d; ++c) {\n      double mx = -INFINITY;\n      for (long j = 0;"),
+    "index_relu_dropped": ("acc += ld(w, dt, (size_t)r * HI + h) * (dot > 0.0 ? dot : 0.0);",
+                           "acc += ld(w, dt, (size_t)r * HI + h) * dot;"),
+    "index_head_weight_dropped": ("acc += ld(w, dt, (size_t)r * HI + h) * (dot > 0.0 ? dot : 0.0);",
+                                  "acc += (dot > 0.0 ? dot : 0.0);"),
+    "index_visibility_off_by_one": ("    vis[r] = (t + 1) / 4;\n", "    vis[r] = t / 4;\n"),
+    "topk_ties_to_higher_index": ("return (a->i < b->i) ? -1 : (a->i > b->i);",
+                                  "return (a->i > b->i) ? -1 : (a->i < b->i);"),
+    "topk_output_unsorted": ("qsort(orow, (size_t)take, sizeof(int32_t), cmp_i32);", ""),
+    "attend_scale": ("scale = 1.0 / sqrt((double)d);", "scale = 1.0 / (double)d;"),
+    "attend_window_off_by_one": ("long w0 = t - window + 1;", "long w0 = t - window + 2;"),
+    "attend_visibility": ("long vis = (t + 1) / m;", "long vis = (t + 2) / m;"),
+    "attend_invisible_index_used": ("if (i < 0 || i >= vis) continue;", "if (i < 0 || i >= nc_max) continue;"),
+    "round_double_rounding": ("r = nearbyint(ldexp(a, -q));", "r = nearbyint(ldexp((double)(float)a, -q));"),
+}
+
+
+def _run_mutant(name, tmpdir):
+    old, new = MUTANTS[name]
+    src = open(SRC).read()
+    assert src.count(old) >= 1, f"mutation {name} no longer applies"
+    mutated = src.replace(old, new, 1)
+    cpath = os.path.join(tmpdir, f"{name}.c")
+    lib = os.path.join(tmpdir, f"lib_{name}.so")
+    with open(cpath, "w") as f:
+        f.write(mutated)
+    subprocess.run(["gcc", "-O2", "-std=c11", "-fopenmp", "-fPIC", "-shared", cpath, "-o", lib, "-lm"],
+                   check=True, capture_output=True)
+    env = dict(os.environ, CSA_ORACLE_LIB=lib, OMP_NUM_THREADS="1")
+    p = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider", *PINS],
+                       cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
+    return name, p.returncode
+
+
+def test_every_planted_mistake_fails_a_pin():
+    with tempfile.TemporaryDirectory() as tmp:
+        with ThreadPoolExecutor(max_workers=max(1, min(8, os.cpu_count() or 1))) as ex:
+            results = list(ex.map(lambda n: _run_mutant(n, tmp), MUTANTS))
+    survivors = [n for n, rc in results if rc == 0]
+    assert not survivors, f"mutants not caught by any pin: {survivors}"
