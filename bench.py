@@ -1,0 +1,354 @@
+#!/usr/bin/env python
+"""Benchmark of the CSA decode step at 1M context on B200.
+
+Workload (default): B=4 sequences of 1,048,576 tokens -> 262,144 compressed
+entries each; 64 query heads x 128, one shared KV head, indexer 64 x 128 with
+bf16 keys, top-k 1024, window 128; seeded synthetic inputs with one planted
+needle per sequence.  A step is one decode step of the whole batch: indexer
+scores over every visible entry, per-query top-k, and attention over the
+selected entries plus the window (the caches are pre-built, as the workload
+states).  The metric is decode queries/s (one query = one sequence's step).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+For N > 1 launch with torchrun; each rank runs its own copy of the batch
+(sequences are independent: no collective on the data path), timing is the
+max over ranks.  `--impl reference` times the CPU oracle (fp64) instead.
+"""
+import argparse
+import datetime
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads as W  # noqa: E402
+
+METRIC = "CSA/HCA decode queries/s at 1M ctx; achieved HBM GB/s as % of B200 peak"
+UNIT = "queries/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "source": "fallback"}
+NOMINAL_HBM_GBS = 8000.0
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=500)
+    p.add_argument("--warmup", type=int, default=20)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--cpu-steps", type=int, default=1, help="oracle steps for cpu_baseline")
+    return p.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            pk = json.load(f)
+        pk["source"] = "measured"
+        return pk
+    return dict(FALLBACK_PEAKS)
+
+
+# --------------------------------------------------------------------------
+# algorithmic bytes (what the method must touch), per query of workload 4
+# --------------------------------------------------------------------------
+def algorithmic_bytes(s):
+    """Bytes per query: the full indexer-key scan, the gathered k entries and
+    window rows, and the query-side vectors (q, indexer queries, head
+    weights) plus the output."""
+    e = 2  # bf16
+    keys = s["nc"] * s["dI"] * e
+    gather = (s["k"] + s["window"]) * s["d"] * e
+    vecs = (s["H"] * s["d"] + s["HI"] * s["dI"] + s["HI"]) * e + s["H"] * s["d"] * e
+    return keys, gather, vecs
+
+
+def scoring_kernel_bytes(s, B):
+    """Per launch of the scoring kernel: keys + indexer queries + head
+    weights read, fp32 scores written."""
+    return B * (s["nc"] * s["dI"] * 2 + s["HI"] * s["dI"] * 2 + s["HI"] * 2 + s["nc"] * 4)
+
+
+# --------------------------------------------------------------------------
+# clocks during the timed region
+# --------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu_id), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for ln in f:
+                parts = [p.strip() for p in ln.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(rows)}
+
+
+def max_over_ranks(vals, world, device):
+    """Element-wise max of per-rank timings (the slowest rank sets the job's
+    time)."""
+    if world <= 1:
+        return list(vals)
+    import torch
+    t = torch.tensor(vals, dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
+
+
+# --------------------------------------------------------------------------
+# the GPU arm
+# --------------------------------------------------------------------------
+def run_ours(args, rank, world, dev):
+    import torch
+    import compressed_sparse_long_03_b200 as csa
+    from tests.helpers import to_dev
+
+    torch.cuda.set_device(dev)
+    wl = W.make(4)
+    s = dict(wl.sizes)
+    B, nc, k, window = s["B"], s["nc"], s["k"], s["window"]
+    D = {n: to_dev(wl[n], f"cuda:{dev}") for n in ("kI", "kv", "win", "q", "qI", "w", "lens")}
+    scores = torch.empty(B, 1, nc, dtype=torch.float32, device=dev)
+    idx = torch.empty(B, 1, k, dtype=torch.int32, device=dev)
+    out = torch.empty(B, 1, s["H"], s["d"], dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        csa.csa_index_scores(D["qI"], D["w"], D["kI"], D["lens"], scores_out=scores)
+        if ev is not None:
+            ev[1].record(stream)
+        csa.csa_topk(scores, D["lens"], k, idx_out=idx)
+        if ev is not None:
+            ev[2].record(stream)
+        csa.csa_attend(D["q"], D["kv"], D["win"], idx, D["lens"], window=window, out=out)
+        if ev is not None:
+            ev[3].record(stream)
+
+    launches_per_step = 3
+    for _ in range(args.warmup):
+        step()
+    csa.check_device_error()
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+
+    K = args.steps
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(f"GPU-{torch.cuda.get_device_properties(dev).uuid}")
+    if rank == 0:
+        sampler.start()
+    barrier()
+    torch.cuda.synchronize()
+    t0.record(stream)
+    for i in range(K):
+        step(evs[i])
+    t1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    clocks = sampler.stop() if rank == 0 else None
+    csa.check_device_error()
+    ms = t0.elapsed_time(t1) / K
+    stage = {name: [evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(K)]
+             for j, name in enumerate(("index_scores", "topk", "attend"))}
+
+    # end to end through the public API from pinned host buffers: H2D of the
+    # step's query inputs, the three calls, D2H of the output
+    host = {n: torch.from_numpy(np.ascontiguousarray(wl[n]).view(np.int16)).pin_memory()
+            for n in ("q", "qI", "w")}
+    out_h = torch.empty(out.shape, dtype=torch.bfloat16).pin_memory()
+    qd = {n: D[n] for n in ("q", "qI", "w")}
+
+    def step_e2e():
+        for n in ("q", "qI", "w"):
+            qd[n].view(torch.int16).copy_(host[n], non_blocking=True)
+        step()
+        out_h.copy_(out, non_blocking=True)
+
+    h2d = sum(host[n].numel() * 2 for n in host)
+    d2h = out_h.numel() * 2
+    for _ in range(3):
+        step_e2e()
+    Ke = max(10, K // 2)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(Ke):
+        step_e2e()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    ms_e2e = e0.elapsed_time(e1) / Ke
+
+    ms, ms_e2e = max_over_ranks([ms, ms_e2e], world, f"cuda:{dev}")
+    return dict(ms=ms, ms_e2e=ms_e2e, stage=stage, clocks=clocks, s=s, B=B, h2d=h2d, d2h=d2h,
+                launches=launches_per_step * K, wl=wl)
+
+
+# --------------------------------------------------------------------------
+# the oracle (CPU) arm
+# --------------------------------------------------------------------------
+def oracle_query_step(wl, b):
+    import oracle
+    s = wl.sizes
+    sl = slice(b, b + 1)
+    idx, _ = oracle.index_topk(wl["qI"][sl], wl["w"][sl], wl["kI"][sl], wl["lens"][sl], s["k"])
+    oracle.attend(wl["q"][sl], wl["kv"][sl], wl["win"][sl], wl["lens"][sl], idx=idx,
+                  window=s["window"])
+
+
+def cpu_baseline(wl, steps=1):
+    """The oracle as it stands on the host cores: `steps` full decode steps
+    of the batch (every query scores all 262,144 entries in fp64)."""
+    import oracle
+    cores = os.cpu_count() or 1
+    oracle.set_threads(cores)
+    B = wl.sizes["B"]
+    t = time.perf_counter()
+    for _ in range(steps):
+        for b in range(B):
+            oracle_query_step(wl, b)
+    dt = time.perf_counter() - t
+    return {"value": steps * B / dt, "unit": UNIT, "cores": oracle.get_threads(), "kind": "oracle",
+            "sample": f"{steps} full decode step(s) of the B={B} batch ({steps * B} queries, "
+                      f"fp64 C oracle, OpenMP)"}
+
+
+def config_block(s, world):
+    return {"workload": "csa_decode_bf16_b4_n1048576", "B": s["B"], "context": s["n"],
+            "entries": s["nc"], "H": s["H"], "d": s["d"], "HI": s["HI"], "dI": s["dI"],
+            "k": s["k"], "window": s["window"],
+            "l2": "inputs larger than L2: the 256 MiB indexer-key cache is re-scanned every step",
+            "parallelism": f"{world} independent replica(s), one per GPU"}
+
+
+def main():
+    args = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.gpus != world and world > 1:
+        print(f"warning: --gpus {args.gpus} but WORLD_SIZE={world}", file=sys.stderr)
+
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        wl = W.make(4)
+        import oracle
+        oracle.set_threads(os.cpu_count() or 1)
+        B = wl.sizes["B"]
+        for i in range(args.warmup):
+            oracle_query_step(wl, i % B)
+        t = time.perf_counter()
+        for i in range(args.steps):
+            oracle_query_step(wl, i % B)
+        dt = time.perf_counter() - t
+        value = args.steps / dt
+        line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+                "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": 1000 * dt / args.steps, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+                "config": config_block(wl.sizes, 1),
+                "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle.get_threads(),
+                                 "kind": "oracle",
+                                 "sample": "one query (one sequence's decode step) per step, "
+                                           "rotating over the batch"},
+                "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}}
+        print(json.dumps(line))
+        return 0
+
+    import torch
+    if world > 1:
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                             device_id=torch.device(f"cuda:{local}"))
+    r = run_ours(args, rank, world, local)
+    s, B = r["s"], r["B"]
+    peaks = load_peaks()
+    hbm_peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    keys, gather, vecs = algorithmic_bytes(s)
+    step_bytes = B * (keys + gather + vecs)
+    value = world * B * 1000.0 / r["ms"]
+    e2e = world * B * 1000.0 / r["ms_e2e"]
+    sc_us = [1000 * x for x in r["stage"]["index_scores"]]
+    sc_avg_s = statistics.mean(sc_us) * 1e-6
+    kb = scoring_kernel_bytes(s, B)
+    achieved = kb / sc_avg_s / 1e9
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": r["ms"], "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded PCG64, planted needles)",
+        "config": config_block(s, world),
+        "hbm": {"algorithmic_bytes_per_step": step_bytes,
+                "achieved_gbs": step_bytes / (r["ms"] * 1e-3) / 1e9,
+                "frac_of_measured": step_bytes / (r["ms"] * 1e-3) / 1e9 / hbm_peak,
+                "frac_of_nominal_8tbs": step_bytes / (r["ms"] * 1e-3) / 1e9 / NOMINAL_HBM_GBS},
+        "roofline": {"kernel": "index_scores", "bound": "hbm", "achieved": achieved,
+                     "peak": hbm_peak, "unit": "GB/s", "frac": achieved / hbm_peak,
+                     "traffic": None, "bytes_per_launch": kb, "peak_source": peaks["source"]},
+        "stages_us": {k: statistics.median(1000 * x for x in v) for k, v in r["stage"].items()},
+        "e2e": {"value": e2e, "unit": UNIT, "h2d_bytes_per_step": r["h2d"],
+                "d2h_bytes_per_step": r["d2h"]},
+        "gpu_launches": r["launches"],
+        "clocks": r["clocks"],
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(r["wl"], args.cpu_steps)
+    if rank == 0:
+        print(json.dumps(line))
+    if world > 1:
+        torch.distributed.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,205 @@
+"""B200 (sm_100a) Compressed Sparse Attention / Heavily Compressed Attention.
+
+A thin ctypes binding of ``libcsa.so`` (declared in ``include/csa.h``).  Each
+function marshals PyTorch CUDA tensors into the C call of the same name; every
+step of the computation runs in the library's CUDA kernels.  PyTorch provides
+device memory and streams only.  There is no CPU path: if the library is not
+built, or a tensor is not a contiguous CUDA tensor, the call raises.
+
+Entry points (method definitions are stated in ``include/csa.h``):
+  csa_compress    CSA overlapping compressor (stride 4, 8-token windows)
+  hca_compress    HCA compressor (stride m, no overlap)
+  csa_index_topk  lightning-indexer scores + per-query top-k
+  csa_attend      MQA attention over the selected entries + sliding window
+  hca_attend      MQA attention over every visible HCA entry + sliding window
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG, "libcsa.so")
+
+F32 = 0
+BF16 = 1
+
+_lib = None
+
+
+class CsaError(RuntimeError):
+    """A library call returned a negative status."""
+
+    def __init__(self, status: int, message: str):
+        super().__init__(f"status {status}: {message}")
+        self.status = status
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libcsa.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing: build it with "
+                              "`python -m compressed_sparse_long_03_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        P, I, F, S = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+        L.csa_version.restype = I
+        L.csa_last_error.restype = ctypes.c_char_p
+        L.csa_check_device_error.argtypes = [P]
+        L.csa_compress.argtypes = [P, P, I, I, I, P, P, P, I, P, P]
+        L.hca_compress.argtypes = [P, P, I, I, I, I, P, P, I, P, P]
+        L.csa_index_topk_workspace_size.argtypes = [I, I, I, I]
+        L.csa_index_topk_workspace_size.restype = S
+        L.csa_index_topk.argtypes = [P, P, P, P, P, I, I, I, I, I, I, I, P, P, P, S, P]
+        L.csa_index_scores.argtypes = [P, P, P, P, P, I, I, I, I, I, I, P, P]
+        L.csa_topk.argtypes = [P, P, P, I, I, I, I, P, P]
+        L.csa_attend.argtypes = [P, P, P, I, P, P, P, I, I, I, I, I, I, I, F, I, P, P]
+        L.hca_attend.argtypes = [P, P, P, I, P, P, I, I, I, I, I, I, I, F, I, P, P]
+        for name in ("csa_check_device_error", "csa_compress", "hca_compress", "csa_index_topk",
+                     "csa_index_scores", "csa_topk", "csa_attend", "hca_attend"):
+            getattr(L, name).restype = I
+        _lib = L
+    return _lib
+
+
+def last_error() -> str:
+    return lib().csa_last_error().decode()
+
+
+def _check(rc: int) -> None:
+    if rc != 0:
+        raise CsaError(rc, last_error())
+
+
+def _dt(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return F32
+    if t.dtype == torch.bfloat16:
+        return BF16
+    raise TypeError(f"float tensors are float32 or bfloat16, got {t.dtype}")
+
+
+def _p(t):
+    """Device pointer of a contiguous CUDA tensor (None -> NULL)."""
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("tensors must live on a CUDA device")
+    if not t.is_contiguous():
+        raise ValueError("tensors must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _s(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _i32(t):
+    if t is not None and t.dtype != torch.int32:
+        raise TypeError("lengths, positions and indices are int32")
+    return _p(t)
+
+
+def check_device_error(stream=None) -> None:
+    """Synchronise the stream and raise if a kernel flagged an invalid length,
+    position or window (the device error word is cleared)."""
+    _check(lib().csa_check_device_error(_s(stream)))
+
+
+def csa_compress(x, lens, W_a, W_b, bias8, out=None, stream=None):
+    """x [B][n_max][d], lens [B] int32, W_a/W_b [d][d], bias8 [8][d]
+    -> [B][ceil(n_max/4)][d] (rows past ceil(lens/4) zero)."""
+    B, n_max, d = x.shape
+    if out is None:
+        out = torch.empty(B, (n_max + 3) // 4, d, dtype=x.dtype, device=x.device)
+    _check(lib().csa_compress(_p(x), _i32(lens), B, n_max, d, _p(W_a), _p(W_b), _p(bias8), _dt(x),
+                              _p(out), _s(stream)))
+    return out
+
+
+def hca_compress(x, lens, W, bias, m=128, out=None, stream=None):
+    """x [B][n_max][d], W [d][d], bias [m][d] -> [B][ceil(n_max/m)][d]."""
+    B, n_max, d = x.shape
+    if out is None:
+        out = torch.empty(B, (n_max + m - 1) // m, d, dtype=x.dtype, device=x.device)
+    _check(lib().hca_compress(_p(x), _i32(lens), B, n_max, d, m, _p(W), _p(bias), _dt(x), _p(out),
+                              _s(stream)))
+    return out
+
+
+def index_topk_workspace_size(B, Tq, nc_max, has_scores_out=False) -> int:
+    return int(lib().csa_index_topk_workspace_size(B, Tq, nc_max, int(bool(has_scores_out))))
+
+
+def csa_index_topk(q_idx, w, k_idx, lens, k, q_pos=None, idx_out=None, scores_out=None,
+                   workspace=None, stream=None):
+    """q_idx [B][Tq][HI][dI], w [B][Tq][HI], k_idx [B][nc_max][dI]
+    -> idx [B][Tq][k] int32 (ascending, -1 padded); fills scores_out
+    [B][Tq][nc_max] float32 when given."""
+    B, Tq, HI, dI = q_idx.shape
+    nc_max = k_idx.shape[1]
+    if idx_out is None:
+        idx_out = torch.empty(B, Tq, k, dtype=torch.int32, device=q_idx.device)
+    need = index_topk_workspace_size(B, Tq, nc_max, scores_out is not None)
+    if workspace is None and need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q_idx.device)
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check(lib().csa_index_topk(_p(q_idx), _p(w), _p(k_idx), _i32(lens), _i32(q_pos), B, Tq, HI, dI,
+                                nc_max, k, _dt(q_idx), _i32(idx_out), _p(scores_out), _p(workspace),
+                                ws_bytes, _s(stream)))
+    return idx_out
+
+
+def csa_index_scores(q_idx, w, k_idx, lens, q_pos=None, scores_out=None, stream=None):
+    """Indexer scores only -> scores [B][Tq][nc_max] float32 (-inf where
+    not visible)."""
+    B, Tq, HI, dI = q_idx.shape
+    nc_max = k_idx.shape[1]
+    if scores_out is None:
+        scores_out = torch.empty(B, Tq, nc_max, dtype=torch.float32, device=q_idx.device)
+    _check(lib().csa_index_scores(_p(q_idx), _p(w), _p(k_idx), _i32(lens), _i32(q_pos), B, Tq, HI, dI,
+                                  nc_max, _dt(q_idx), _p(scores_out), _s(stream)))
+    return scores_out
+
+
+def csa_topk(scores, lens, k, q_pos=None, idx_out=None, stream=None):
+    """Top-k selection over given scores [B][Tq][nc_max] -> idx [B][Tq][k]."""
+    B, Tq, nc_max = scores.shape
+    if scores.dtype != torch.float32:
+        raise TypeError("scores are float32")
+    if idx_out is None:
+        idx_out = torch.empty(B, Tq, k, dtype=torch.int32, device=scores.device)
+    _check(lib().csa_topk(_p(scores), _i32(lens), _i32(q_pos), B, Tq, nc_max, k, _i32(idx_out),
+                          _s(stream)))
+    return idx_out
+
+
+def csa_attend(q, kv_c, kv_tok, idx, lens, q_pos=None, window=128, scale=0.0, out=None,
+               stream=None):
+    """q [B][Tq][H][d], kv_c [B][nc_max][d], kv_tok [B][n_tok][d] (ring),
+    idx [B][Tq][k] -> out [B][Tq][H][d]."""
+    B, Tq, H, d = q.shape
+    if out is None:
+        out = torch.empty_like(q)
+    _check(lib().csa_attend(_p(q), _p(kv_c), _p(kv_tok), kv_tok.shape[1], _i32(idx), _i32(lens),
+                            _i32(q_pos), B, Tq, H, d, kv_c.shape[1], idx.shape[-1], window,
+                            float(scale), _dt(q), _p(out), _s(stream)))
+    return out
+
+
+def hca_attend(q, kv_c, kv_tok, lens, q_pos=None, m=128, window=128, scale=0.0, out=None,
+               stream=None):
+    """q [B][Tq][H][d], kv_c [B][nc_max][d], kv_tok [B][n_tok][d] (ring)
+    -> out [B][Tq][H][d]."""
+    B, Tq, H, d = q.shape
+    if out is None:
+        out = torch.empty_like(q)
+    _check(lib().hca_attend(_p(q), _p(kv_c), _p(kv_tok), kv_tok.shape[1], _i32(lens), _i32(q_pos),
+                            B, Tq, H, d, kv_c.shape[1], m, window, float(scale), _dt(q), _p(out),
+                            _s(stream)))
+    return out

@@ -1,0 +1,49 @@
+"""Build libcsa.so (the C-ABI library of include/csa.h) for sm_100a, in-tree.
+
+    python -m compressed_sparse_long_03_b200.build [--force]
+
+nvcc cross-compiles for sm_100a without a GPU, so this runs on any host with
+CUDA 12.9.  The library is one translation unit (csrc/csa_api.cu includes the
+kernel headers).
+"""
+import os
+import subprocess
+import sys
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+ROOT = os.path.dirname(PKG)
+CSRC = os.path.join(PKG, "csrc")
+INCLUDE = os.path.join(ROOT, "include")
+LIB = os.path.join(PKG, "libcsa.so")
+NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
+
+NVCC_FLAGS = [
+    "-O3", "-std=c++17", "-lineinfo",
+    "-gencode", "arch=compute_100a,code=sm_100a",
+    "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",
+    "--expt-relaxed-constexpr",
+]
+
+
+def _sources():
+    return [os.path.join(CSRC, f) for f in sorted(os.listdir(CSRC))
+            if f.endswith((".cu", ".cuh", ".h"))] + [os.path.join(INCLUDE, "csa.h")]
+
+
+def build(force: bool = False, verbose: bool = False, extra_flags=()) -> str:
+    srcs = _sources()
+    if (not force and os.path.exists(LIB)
+            and os.path.getmtime(LIB) >= max(os.path.getmtime(s) for s in srcs)):
+        return LIB
+    cmd = [NVCC, *NVCC_FLAGS, *extra_flags, "-I", INCLUDE, "-I", CSRC, "-shared",
+           os.path.join(CSRC, "csa_api.cu"), "-o", LIB + ".tmp", "-lcuda"]
+    if verbose:
+        print(" ".join(cmd))
+    subprocess.run(cmd, check=True)
+    os.replace(LIB + ".tmp", LIB)
+    return LIB
+
+
+if __name__ == "__main__":
+    print(build(force="--force" in sys.argv, verbose=True,
+                extra_flags=["-Xptxas", "-v"] if "--ptxas-v" in sys.argv else []))

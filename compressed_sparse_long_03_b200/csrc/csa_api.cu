@@ -1,0 +1,453 @@
+// csa_api.cu -- the C ABI (include/csa.h): host-side validation, launch
+// configuration and error reporting for the CSA / HCA kernels.
+//
+// The whole library is this one translation unit: every kernel header is
+// included here, so the device error word has one definition and no device
+// linking is needed.
+#include <cuda_runtime.h>
+
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+#include <unordered_map>
+
+#include "csa.h"
+
+#include "common.cuh"
+#include "compress.cuh"
+#include "index_score_fma.cuh"
+#include "topk.cuh"
+#include "attend_fma.cuh"
+
+namespace {
+
+thread_local std::string g_last_error;
+
+int fail(int code, const char *fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return code;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int launch_status(const char *what) {
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(CSA_ERR_LAUNCH, "%s: launch failed: %s", what, cudaGetErrorString(e));
+  return CSA_OK;
+}
+
+// Raise a kernel's dynamic shared-memory limit once per (kernel, device).
+std::mutex g_attr_mu;
+std::unordered_map<std::string, size_t> g_attr_done;
+
+template <typename K>
+int ensure_smem(K kernel, size_t bytes, const char *what) {
+  if (bytes <= 48 * 1024) return CSA_OK;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return fail(CSA_ERR_CUDA, "%s: cudaGetDevice failed", what);
+  char key[64];
+  snprintf(key, sizeof(key), "%p/%d", reinterpret_cast<const void *>(kernel), dev);
+  std::lock_guard<std::mutex> lk(g_attr_mu);
+  auto it = g_attr_done.find(key);
+  if (it != g_attr_done.end() && it->second >= bytes) return CSA_OK;
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  if (e != cudaSuccess)
+    return fail(CSA_ERR_CUDA, "%s: cannot reserve %zu B of shared memory: %s", what, bytes,
+                cudaGetErrorString(e));
+  g_attr_done[key] = bytes;
+  return CSA_OK;
+}
+
+// Launch `kernel` on a 1-D grid of clusters of `cs` CTAs (cs == 1: a plain
+// launch).
+template <typename... KArgs, typename... Args>
+int launch_cluster(void (*kernel)(KArgs...), int cs, unsigned grid, unsigned block, size_t smem,
+                   cudaStream_t stream, const char *what, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid, 1, 1);
+  cfg.blockDim = dim3(block, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  if (cs > 1) {
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = cs;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+  }
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, args...);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return fail(CSA_ERR_LAUNCH, "%s: launch failed: %s", what, cudaGetErrorString(e));
+  }
+  return CSA_OK;
+}
+
+int check_dtype(csa_dtype dt, const char *what) {
+  if (dt != CSA_F32 && dt != CSA_BF16) return fail(CSA_ERR_DTYPE, "%s: unknown dtype %d", what, (int)dt);
+  return CSA_OK;
+}
+
+constexpr int kMaxIndexEntries = csa::kTopkMaxCluster * csa::kTopkSliceCap;  // 393216
+
+int topk_cluster_size(int nc_max) {
+  int cs = 1;
+  while (cs < csa::kTopkMaxCluster && (long)cs * 8192 < nc_max) cs *= 2;
+  while ((long)cs * csa::kTopkSliceCap < nc_max) cs *= 2;  // never beyond the cap (validated)
+  return cs;
+}
+
+int attend_cluster_size(long max_keys) {
+  int cs = 1;
+  while (cs < 8 && (long)cs * 64 * 2 <= max_keys) cs *= 2;
+  return cs;
+}
+
+// ---------------------------------------------------------------------------
+// compressors
+// ---------------------------------------------------------------------------
+template <typename T>
+int launch_csa_compress(const void *x, const int32_t *lens, int B, int n_max, int d, const void *Wa,
+                        const void *Wb, const void *b8, void *out, cudaStream_t st) {
+  const int nc_max = (n_max + 3) / 4;
+  dim3 grid((nc_max + csa::kCsaEntries - 1) / csa::kCsaEntries, B);
+  auto X = static_cast<const T *>(x);
+  auto A = static_cast<const T *>(Wa);
+  auto Bw = static_cast<const T *>(Wb);
+  auto Z = static_cast<const T *>(b8);
+  auto O = static_cast<T *>(out);
+  switch (d) {
+    case 32: csa::k_csa_compress<T, 32><<<grid, 32, 0, st>>>(X, lens, n_max, A, Bw, Z, O, nc_max); break;
+    case 64: csa::k_csa_compress<T, 64><<<grid, 64, 0, st>>>(X, lens, n_max, A, Bw, Z, O, nc_max); break;
+    default: csa::k_csa_compress<T, 128><<<grid, 128, 0, st>>>(X, lens, n_max, A, Bw, Z, O, nc_max); break;
+  }
+  return launch_status("csa_compress");
+}
+
+template <typename T>
+int launch_hca_compress(const void *x, const int32_t *lens, int B, int n_max, int d, int m,
+                        const void *W, const void *bias, void *out, cudaStream_t st) {
+  const int nc_max = (int)(((long)n_max + m - 1) / m);
+  dim3 grid(nc_max, B);
+  auto X = static_cast<const T *>(x);
+  auto Wp = static_cast<const T *>(W);
+  auto Z = static_cast<const T *>(bias);
+  auto O = static_cast<T *>(out);
+  switch (d) {
+    case 32: csa::k_hca_compress<T, 32><<<grid, 32, 0, st>>>(X, lens, n_max, m, Wp, Z, O, nc_max); break;
+    case 64: csa::k_hca_compress<T, 64><<<grid, 64, 0, st>>>(X, lens, n_max, m, Wp, Z, O, nc_max); break;
+    default: csa::k_hca_compress<T, 128><<<grid, 128, 0, st>>>(X, lens, n_max, m, Wp, Z, O, nc_max); break;
+  }
+  return launch_status("hca_compress");
+}
+
+// ---------------------------------------------------------------------------
+// indexer scores + top-k
+// ---------------------------------------------------------------------------
+template <typename T, int DI>
+int launch_index_fma(const void *qI, const void *w, const void *kI, const int32_t *lens,
+                     const int32_t *q_pos, int R, int Tq, int HI, int nc_max, float *scores,
+                     cudaStream_t st) {
+  const int tiles = (nc_max + csa::kIdxFmaTile - 1) / csa::kIdxFmaTile;
+  const size_t smem = sizeof(float) * ((size_t)HI * DI + ((HI + 3) & ~3) +
+                                       (size_t)csa::kIdxFmaTile * (DI + 1));
+  auto kern = csa::k_index_score_fma<T, DI>;
+  int rc = ensure_smem(kern, smem, "csa_index_topk");
+  if (rc) return rc;
+  dim3 grid(tiles, R);
+  kern<<<grid, csa::kIdxFmaTile, smem, st>>>(static_cast<const T *>(qI), static_cast<const T *>(w),
+                                             static_cast<const T *>(kI), lens, q_pos, Tq, HI,
+                                             nc_max, scores);
+  return launch_status("csa_index_topk (scores)");
+}
+
+template <int CS>
+int launch_topk(const float *scores, const int32_t *lens, const int32_t *q_pos, int R, int Tq,
+                int nc_max, int k, int32_t *idx_out, cudaStream_t st) {
+  const int per = (nc_max + CS - 1) / CS;
+  const size_t smem = sizeof(uint32_t) * (size_t)(per > 0 ? per : 1);
+  auto kern = csa::k_topk<CS>;
+  int rc = ensure_smem(kern, smem, "csa_index_topk");
+  if (rc) return rc;
+  return launch_cluster(kern, CS, (unsigned)CS * R, csa::kTopkThreads, smem, st,
+                        "csa_index_topk (select)", scores, lens, q_pos, Tq, nc_max, k, idx_out);
+}
+
+// ---------------------------------------------------------------------------
+// attention
+// ---------------------------------------------------------------------------
+template <typename T, int D>
+int launch_attend_fma(const csa::AttendArgs &a, int R, long max_keys, cudaStream_t st,
+                      const char *what) {
+  const int cs = attend_cluster_size(max_keys);
+  const size_t smem = sizeof(float) * ((size_t)a.H * D + csa::kAttTile * (D + 1) + 2 * a.H) +
+                      sizeof(int) * csa::kAttTile;
+  void (*kern)(csa::AttendArgs) = nullptr;
+  switch (cs) {
+    case 1: kern = csa::k_attend_fma<T, D, 1>; break;
+    case 2: kern = csa::k_attend_fma<T, D, 2>; break;
+    case 4: kern = csa::k_attend_fma<T, D, 4>; break;
+    default: kern = csa::k_attend_fma<T, D, 8>; break;
+  }
+  int rc = ensure_smem(kern, smem, what);
+  if (rc) return rc;
+  return launch_cluster(kern, cs, (unsigned)cs * R, csa::kAttThreads, smem, st, what, a);
+}
+
+int attend_common(const void *q, const void *kv_c, const void *kv_tok, int n_tok,
+                  const int32_t *idx, const int32_t *lens, const int32_t *q_pos, int B, int Tq,
+                  int H, int d, int nc_max, int k, int m, int window, float scale, csa_dtype dt,
+                  void *out, void *stream, const char *what) {
+  int rc = check_dtype(dt, what);
+  if (rc) return rc;
+  if (B < 0 || Tq < 0) return fail(CSA_ERR_SHAPE, "%s: B=%d and Tq=%d must be >= 0", what, B, Tq);
+  if ((long)B * Tq == 0) return CSA_OK;
+  if (!q || !kv_tok || !lens || !out || (idx == nullptr && k > 0) || (nc_max > 0 && !kv_c))
+    return fail(CSA_ERR_NULL, "%s: a required pointer is NULL", what);
+  if (!aligned16(q) || !aligned16(kv_tok) || !aligned16(out) || (kv_c && !aligned16(kv_c)))
+    return fail(CSA_ERR_ALIGN, "%s: tensors must be 16-byte aligned", what);
+  if (d != 64 && d != 128) return fail(CSA_ERR_UNSUPPORTED, "%s: d=%d not in {64,128}", what, d);
+  if (H < 1 || H > 128) return fail(CSA_ERR_UNSUPPORTED, "%s: H=%d not in [1,128]", what, H);
+  if (window < 1 || window > 4096)
+    return fail(CSA_ERR_UNSUPPORTED, "%s: window=%d not in [1,4096]", what, window);
+  if (n_tok < 1) return fail(CSA_ERR_SHAPE, "%s: n_tok=%d must be >= 1", what, n_tok);
+  if (nc_max < 0) return fail(CSA_ERR_SHAPE, "%s: nc_max=%d must be >= 0", what, nc_max);
+  if ((long)B * Tq > (1L << 26)) return fail(CSA_ERR_UNSUPPORTED, "%s: too many query rows", what);
+  csa::AttendArgs a;
+  a.q = q;
+  a.kv_c = kv_c;
+  a.kv_tok = kv_tok;
+  a.idx = idx;
+  a.lens = lens;
+  a.q_pos = q_pos;
+  a.out = out;
+  a.n_tok = n_tok;
+  a.k = k;
+  a.Tq = Tq;
+  a.H = H;
+  a.nc_max = nc_max;
+  a.m = m;
+  a.window = window;
+  const float sc = scale > 0.f ? scale : 1.0f / sqrtf((float)d);
+  a.scale_log2 = sc * 1.4426950408889634f;
+  const int R = B * Tq;
+  const long max_keys = (idx ? (long)k : (long)nc_max) + window;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (dt == CSA_F32)
+    return d == 64 ? launch_attend_fma<float, 64>(a, R, max_keys, st, what)
+                   : launch_attend_fma<float, 128>(a, R, max_keys, st, what);
+  return d == 64 ? launch_attend_fma<__nv_bfloat16, 64>(a, R, max_keys, st, what)
+                 : launch_attend_fma<__nv_bfloat16, 128>(a, R, max_keys, st, what);
+}
+
+}  // namespace
+
+// ===========================================================================
+// extern "C" entry points
+// ===========================================================================
+extern "C" {
+
+int csa_version(void) { return (0 << 16) | 1; }
+
+const char *csa_last_error(void) { return g_last_error.c_str(); }
+
+int csa_check_device_error(void *stream) {
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail(CSA_ERR_CUDA, "stream error: %s", cudaGetErrorString(e));
+  int v = 0;
+  e = cudaMemcpyFromSymbol(&v, csa::g_dev_err, sizeof(int));
+  if (e != cudaSuccess) return fail(CSA_ERR_CUDA, "reading the device error word: %s", cudaGetErrorString(e));
+  if (v == 0) return CSA_OK;
+  const int zero = 0;
+  cudaMemcpyToSymbol(csa::g_dev_err, &zero, sizeof(int));
+  static const char *what[] = {"", "a query position outside its sequence",
+                               "a sequence length outside [0, n_max]",
+                               "visible entries exceed the cache rows",
+                               "a query window larger than the token ring"};
+  return fail(CSA_ERR_DEVICE, "device check failed: %s", (v > 0 && v < 5) ? what[v] : "unknown");
+}
+
+int csa_compress(const void *x, const int32_t *lens, int B, int n_max, int d, const void *W_a,
+                 const void *W_b, const void *bias8, csa_dtype dt, void *out, void *stream) {
+  const char *what = "csa_compress";
+  int rc = check_dtype(dt, what);
+  if (rc) return rc;
+  if (B < 0 || n_max < 0) return fail(CSA_ERR_SHAPE, "%s: B=%d, n_max=%d must be >= 0", what, B, n_max);
+  if (d != 32 && d != 64 && d != 128) return fail(CSA_ERR_UNSUPPORTED, "%s: d=%d not in {32,64,128}", what, d);
+  if (B == 0 || n_max == 0) return CSA_OK;
+  if (B > 65535) return fail(CSA_ERR_UNSUPPORTED, "%s: B=%d > 65535", what, B);
+  if (!x || !lens || !W_a || !W_b || !bias8 || !out) return fail(CSA_ERR_NULL, "%s: a required pointer is NULL", what);
+  if (!aligned16(x) || !aligned16(W_a) || !aligned16(W_b) || !aligned16(bias8) || !aligned16(out))
+    return fail(CSA_ERR_ALIGN, "%s: tensors must be 16-byte aligned", what);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (dt == CSA_F32) return launch_csa_compress<float>(x, lens, B, n_max, d, W_a, W_b, bias8, out, st);
+  return launch_csa_compress<__nv_bfloat16>(x, lens, B, n_max, d, W_a, W_b, bias8, out, st);
+}
+
+int hca_compress(const void *x, const int32_t *lens, int B, int n_max, int d, int m, const void *W,
+                 const void *bias, csa_dtype dt, void *out, void *stream) {
+  const char *what = "hca_compress";
+  int rc = check_dtype(dt, what);
+  if (rc) return rc;
+  if (B < 0 || n_max < 0) return fail(CSA_ERR_SHAPE, "%s: B=%d, n_max=%d must be >= 0", what, B, n_max);
+  if (d != 32 && d != 64 && d != 128) return fail(CSA_ERR_UNSUPPORTED, "%s: d=%d not in {32,64,128}", what, d);
+  if (m < 1 || m > 4096) return fail(CSA_ERR_UNSUPPORTED, "%s: m=%d not in [1,4096]", what, m);
+  if (B == 0 || n_max == 0) return CSA_OK;
+  if (B > 65535) return fail(CSA_ERR_UNSUPPORTED, "%s: B=%d > 65535", what, B);
+  if (!x || !lens || !W || !bias || !out) return fail(CSA_ERR_NULL, "%s: a required pointer is NULL", what);
+  if (!aligned16(x) || !aligned16(W) || !aligned16(bias) || !aligned16(out))
+    return fail(CSA_ERR_ALIGN, "%s: tensors must be 16-byte aligned", what);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (dt == CSA_F32) return launch_hca_compress<float>(x, lens, B, n_max, d, m, W, bias, out, st);
+  return launch_hca_compress<__nv_bfloat16>(x, lens, B, n_max, d, m, W, bias, out, st);
+}
+
+size_t csa_index_topk_workspace_size(int B, int Tq, int nc_max, int has_scores_out) {
+  if (B <= 0 || Tq <= 0 || nc_max <= 0 || has_scores_out) return 0;
+  const size_t bytes = sizeof(float) * (size_t)B * Tq * nc_max;
+  return (bytes + 255) & ~(size_t)255;
+}
+
+}  // extern "C"
+
+namespace {
+
+int index_scores_impl(const void *q_idx, const void *w, const void *k_idx, const int32_t *lens,
+                      const int32_t *q_pos, int B, int Tq, int HI, int dI, int nc_max,
+                      csa_dtype dt, float *scores, cudaStream_t st) {
+  const int R = B * Tq;
+  if (R == 0 || nc_max == 0) return CSA_OK;
+  if (R > 65535) return fail(CSA_ERR_UNSUPPORTED, "csa_index_scores: B*Tq=%d > 65535", R);
+  if (dt == CSA_F32) {
+    switch (dI) {
+      case 32: return launch_index_fma<float, 32>(q_idx, w, k_idx, lens, q_pos, R, Tq, HI, nc_max, scores, st);
+      case 64: return launch_index_fma<float, 64>(q_idx, w, k_idx, lens, q_pos, R, Tq, HI, nc_max, scores, st);
+      default: return launch_index_fma<float, 128>(q_idx, w, k_idx, lens, q_pos, R, Tq, HI, nc_max, scores, st);
+    }
+  }
+  switch (dI) {
+    case 32: return launch_index_fma<__nv_bfloat16, 32>(q_idx, w, k_idx, lens, q_pos, R, Tq, HI, nc_max, scores, st);
+    case 64: return launch_index_fma<__nv_bfloat16, 64>(q_idx, w, k_idx, lens, q_pos, R, Tq, HI, nc_max, scores, st);
+    default: return launch_index_fma<__nv_bfloat16, 128>(q_idx, w, k_idx, lens, q_pos, R, Tq, HI, nc_max, scores, st);
+  }
+}
+
+int topk_impl(const float *scores, const int32_t *lens, const int32_t *q_pos, int B, int Tq,
+              int nc_max, int k, int32_t *idx_out, cudaStream_t st) {
+  const int R = B * Tq;
+  if (R == 0) return CSA_OK;
+  switch (topk_cluster_size(nc_max)) {
+    case 1: return launch_topk<1>(scores, lens, q_pos, R, Tq, nc_max, k, idx_out, st);
+    case 2: return launch_topk<2>(scores, lens, q_pos, R, Tq, nc_max, k, idx_out, st);
+    case 4: return launch_topk<4>(scores, lens, q_pos, R, Tq, nc_max, k, idx_out, st);
+    default: return launch_topk<8>(scores, lens, q_pos, R, Tq, nc_max, k, idx_out, st);
+  }
+}
+
+// shared argument checks of the indexer entry points
+int check_index_args(const char *what, csa_dtype dt, int B, int Tq, int HI, int dI, int nc_max) {
+  int rc = check_dtype(dt, what);
+  if (rc) return rc;
+  if (B < 0 || Tq < 0 || nc_max < 0) return fail(CSA_ERR_SHAPE, "%s: B, Tq, nc_max must be >= 0", what);
+  if (HI < 1 || HI > 128) return fail(CSA_ERR_UNSUPPORTED, "%s: HI=%d not in [1,128]", what, HI);
+  if (dI != 32 && dI != 64 && dI != 128) return fail(CSA_ERR_UNSUPPORTED, "%s: dI=%d not in {32,64,128}", what, dI);
+  if (nc_max > kMaxIndexEntries)
+    return fail(CSA_ERR_UNSUPPORTED, "%s: nc_max=%d > %d", what, nc_max, kMaxIndexEntries);
+  if ((long)B * Tq > 65535) return fail(CSA_ERR_UNSUPPORTED, "%s: B*Tq=%ld > 65535", what, (long)B * Tq);
+  return CSA_OK;
+}
+
+int check_topk_args(const char *what, int B, int Tq, int nc_max, int k) {
+  if (B < 0 || Tq < 0 || nc_max < 0) return fail(CSA_ERR_SHAPE, "%s: B, Tq, nc_max must be >= 0", what);
+  if (k < 1 || k > 4096) return fail(CSA_ERR_UNSUPPORTED, "%s: k=%d not in [1,4096]", what, k);
+  if (nc_max > kMaxIndexEntries)
+    return fail(CSA_ERR_UNSUPPORTED, "%s: nc_max=%d > %d", what, nc_max, kMaxIndexEntries);
+  if ((long)B * Tq > 65535) return fail(CSA_ERR_UNSUPPORTED, "%s: B*Tq=%ld > 65535", what, (long)B * Tq);
+  return CSA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int csa_index_scores(const void *q_idx, const void *w, const void *k_idx, const int32_t *lens,
+                     const int32_t *q_pos, int B, int Tq, int HI, int dI, int nc_max,
+                     csa_dtype dt, float *scores_out, void *stream) {
+  const char *what = "csa_index_scores";
+  int rc = check_index_args(what, dt, B, Tq, HI, dI, nc_max);
+  if (rc) return rc;
+  if ((long)B * Tq == 0 || nc_max == 0) return CSA_OK;
+  if (!q_idx || !w || !k_idx || !lens || !scores_out)
+    return fail(CSA_ERR_NULL, "%s: a required pointer is NULL", what);
+  if (!aligned16(q_idx) || !aligned16(w) || !aligned16(k_idx) || !aligned16(scores_out))
+    return fail(CSA_ERR_ALIGN, "%s: tensors must be 16-byte aligned", what);
+  return index_scores_impl(q_idx, w, k_idx, lens, q_pos, B, Tq, HI, dI, nc_max, dt, scores_out,
+                           static_cast<cudaStream_t>(stream));
+}
+
+int csa_topk(const float *scores, const int32_t *lens, const int32_t *q_pos, int B, int Tq,
+             int nc_max, int k, int32_t *idx_out, void *stream) {
+  const char *what = "csa_topk";
+  int rc = check_topk_args(what, B, Tq, nc_max, k);
+  if (rc) return rc;
+  if ((long)B * Tq == 0) return CSA_OK;
+  if (!lens || !idx_out || (nc_max > 0 && !scores)) return fail(CSA_ERR_NULL, "%s: a required pointer is NULL", what);
+  if (scores && !aligned16(scores)) return fail(CSA_ERR_ALIGN, "%s: scores must be 16-byte aligned", what);
+  return topk_impl(scores, lens, q_pos, B, Tq, nc_max, k, idx_out, static_cast<cudaStream_t>(stream));
+}
+
+int csa_index_topk(const void *q_idx, const void *w, const void *k_idx, const int32_t *lens,
+                   const int32_t *q_pos, int B, int Tq, int HI, int dI, int nc_max, int k,
+                   csa_dtype dt, int32_t *idx_out, float *scores_out, void *workspace,
+                   size_t ws_bytes, void *stream) {
+  const char *what = "csa_index_topk";
+  int rc = check_index_args(what, dt, B, Tq, HI, dI, nc_max);
+  if (rc) return rc;
+  rc = check_topk_args(what, B, Tq, nc_max, k);
+  if (rc) return rc;
+  if ((long)B * Tq == 0) return CSA_OK;
+  if (!q_idx || !w || !lens || !idx_out || (nc_max > 0 && !k_idx))
+    return fail(CSA_ERR_NULL, "%s: a required pointer is NULL", what);
+  if (!aligned16(q_idx) || !aligned16(w) || (k_idx && !aligned16(k_idx)) ||
+      (scores_out && !aligned16(scores_out)))
+    return fail(CSA_ERR_ALIGN, "%s: tensors must be 16-byte aligned", what);
+  const size_t need = csa_index_topk_workspace_size(B, Tq, nc_max, scores_out != nullptr);
+  if (need > 0 && (!workspace || ws_bytes < need))
+    return fail(CSA_ERR_WORKSPACE, "%s: workspace of %zu B needed, %zu given", what, need,
+                workspace ? ws_bytes : (size_t)0);
+  if (need > 0 && !aligned16(workspace)) return fail(CSA_ERR_ALIGN, "%s: workspace must be 16-byte aligned", what);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  float *scores = scores_out ? scores_out : static_cast<float *>(workspace);
+  rc = index_scores_impl(q_idx, w, k_idx, lens, q_pos, B, Tq, HI, dI, nc_max, dt, scores, st);
+  if (rc) return rc;
+  return topk_impl(scores, lens, q_pos, B, Tq, nc_max, k, idx_out, st);
+}
+
+int csa_attend(const void *q, const void *kv_c, const void *kv_tok, int n_tok, const int32_t *idx,
+               const int32_t *lens, const int32_t *q_pos, int B, int Tq, int H, int d, int nc_max,
+               int k, int window, float scale, csa_dtype dt, void *out, void *stream) {
+  if (k < 1 || k > 4096) return fail(CSA_ERR_UNSUPPORTED, "csa_attend: k=%d not in [1,4096]", k);
+  if (!idx && (long)B * Tq > 0) return fail(CSA_ERR_NULL, "csa_attend: idx is NULL");
+  return attend_common(q, kv_c, kv_tok, n_tok, idx, lens, q_pos, B, Tq, H, d, nc_max, k, 4, window,
+                       scale, dt, out, stream, "csa_attend");
+}
+
+int hca_attend(const void *q, const void *kv_c, const void *kv_tok, int n_tok,
+               const int32_t *lens, const int32_t *q_pos, int B, int Tq, int H, int d, int nc_max,
+               int m, int window, float scale, csa_dtype dt, void *out, void *stream) {
+  if (m < 1 || m > 4096) return fail(CSA_ERR_UNSUPPORTED, "hca_attend: m=%d not in [1,4096]", m);
+  if (nc_max > 65536) return fail(CSA_ERR_UNSUPPORTED, "hca_attend: nc_max=%d > 65536", nc_max);
+  return attend_common(q, kv_c, kv_tok, n_tok, nullptr, lens, q_pos, B, Tq, H, d, nc_max, 0, m,
+                       window, scale, dt, out, stream, "hca_attend");
+}
+
+}  // extern "C"

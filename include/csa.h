@@ -1,0 +1,226 @@
+/*
+ * csa.h -- C ABI of the B200 (sm_100a) Compressed Sparse Attention (CSA) /
+ * Heavily Compressed Attention (HCA) decode/prefill hot path.
+ *
+ * The method (DeepSeek-V4's million-token attention) is described in prose
+ * on "Anatomy of a Frontier Model: Reading DeepSeek-V4 Through Part V",
+ * section "The attention: compress, then select" (CSA and HCA bullets, and
+ * the three details that follow them) and section "The skeleton, and what's
+ * kept"; on "The Exchange Rates of a Million Tokens", section 3 ("Rate #2");
+ * and on "DeepSeek V4: How It Made Million-Token AI", section "The Memory
+ * Problem Nobody Wanted to Solve".  Each entry point below cites the passage
+ * it realises and states the reading taken where the prose leaves a step
+ * open.
+ *
+ * Conventions shared by every entry point
+ *  - Pointers are DEVICE pointers owned by the caller.  The library allocates
+ *    no device memory; where scratch is needed the caller passes a workspace
+ *    sized by the matching *_workspace_size query.
+ *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy
+ *    default stream).  A return of CSA_OK means the work was enqueued.
+ *  - Tensors are dense, row-major, with the innermost dimension contiguous;
+ *    every float tensor pointer must be 16-byte aligned.  `dt` gives the
+ *    element type of every float tensor of the call (CSA_F32: float;
+ *    CSA_BF16: bfloat16); lengths, positions and indices are int32.
+ *  - Arithmetic is fp32 (bf16 inputs are multiplied on the tensor cores with
+ *    fp32 accumulation); outputs are rounded to `dt`, nearest-even.
+ *  - Arguments are validated on the host before anything is launched; a
+ *    failing call returns a negative status, launches nothing and leaves a
+ *    message for csa_last_error().  Values that live in device memory
+ *    (lengths, positions, indices) are checked by the kernels: an invalid
+ *    query writes a zero output row and raises the device error word, read
+ *    (and cleared) by csa_check_device_error().  Nothing traps or exits.
+ *  - Query positions: q_pos[b][tq] is the 0-based position t of query
+ *    (b, tq) in sequence b; with q_pos == NULL, t = lens[b] - Tq + tq (the
+ *    last Tq tokens: t = lens[b]-1 for a decode step).  Valid: 0 <= t <
+ *    lens[b].
+ *  - Visibility ("three details": an entry is formed only once its block is
+ *    complete): a query at position t sees compressed entries
+ *    i < floor((t+1)/m) (m = 4 for CSA), plus the window tokens
+ *    max(0, t-window+1) .. t.
+ */
+#ifndef CSA_B200_H
+#define CSA_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define CSA_API __attribute__((visibility("default")))
+#else
+#define CSA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum { CSA_F32 = 0, CSA_BF16 = 1 } csa_dtype;
+
+/* status codes */
+#define CSA_OK 0
+#define CSA_ERR_NULL (-1)        /* a required pointer is NULL                    */
+#define CSA_ERR_ALIGN (-2)       /* a tensor pointer is not 16-byte aligned       */
+#define CSA_ERR_SHAPE (-3)       /* a size is out of range or inconsistent        */
+#define CSA_ERR_DTYPE (-4)       /* dt is not a csa_dtype                         */
+#define CSA_ERR_UNSUPPORTED (-5) /* outside the supported set (see each call)     */
+#define CSA_ERR_WORKSPACE (-6)   /* workspace NULL or smaller than required       */
+#define CSA_ERR_LAUNCH (-7)      /* a kernel launch failed                        */
+#define CSA_ERR_DEVICE (-8)      /* a kernel found an invalid length/position     */
+#define CSA_ERR_CUDA (-9)        /* another CUDA runtime call failed              */
+
+/* Library version, (major << 16) | minor. */
+CSA_API int csa_version(void);
+
+/* Message describing the last failing call on this host thread ("" if none).
+ * The string is owned by the library and valid until the next call on the
+ * same thread. */
+CSA_API const char *csa_last_error(void);
+
+/* Synchronise `stream`, then return CSA_ERR_DEVICE if any kernel of this
+ * library on the current device has raised the device error word since the
+ * last check (clearing it), else CSA_OK.  CSA_ERR_CUDA if the stream itself
+ * reports an error. */
+CSA_API int csa_check_device_error(void *stream);
+
+/* ------------------------------------------------------------------------
+ * csa_compress -- CSA overlapping compressor (stride 4, 8-token windows).
+ *
+ * Anatomy page, CSA bullet: every 4 tokens become one cache entry, a learned
+ * softmax-weighted pooling of their key-value vectors computed per channel
+ * with learned position biases; each entry pools 8 tokens, its own block and
+ * the one before.  Exchange Rates page, section 3: two series C^a / C^b
+ * overlapping across block boundaries under one joint softmax.  Reading:
+ * entry i pools tokens s = 4(i-1)+j, j = 0..7; slots j < 4 (block i-1) use
+ * W_a, slots j >= 4 (block i) use W_b:
+ *     z_s[c] = sum_e x_s[e] W[e][c] + bias8[j][c]
+ *     out_i[c] = sum_s softmax_s(z_s[c]) x_s[c]
+ * over the tokens with 0 <= s < lens[b] (others masked: entry 0 pools 4
+ * tokens, a trailing partial block pools what exists).  The same call builds
+ * the indexer-key cache from per-token indexer keys with their own params.
+ *
+ *   x      [B][n_max][d]   per-token key-value vectors (or indexer keys)
+ *   lens   [B]             tokens of each sequence, 0 <= lens[b] <= n_max
+ *   W_a,W_b [d][d]         logit weights, indexed [in][out]
+ *   bias8  [8][d]          position biases
+ *   out    [B][ceil(n_max/4)][d]; rows i >= ceil(lens[b]/4) are set to 0.
+ * Supported: d in {32, 64, 128}; B >= 0, n_max >= 0.
+ * ---------------------------------------------------------------------- */
+CSA_API int csa_compress(const void *x, const int32_t *lens, int B, int n_max, int d, const void *W_a,
+                 const void *W_b, const void *bias8, csa_dtype dt, void *out, void *stream);
+
+/* ------------------------------------------------------------------------
+ * hca_compress -- HCA compressor (stride m, no overlap).
+ *
+ * Anatomy page, HCA bullet: every 128 tokens become one entry, without
+ * overlap; Million-Token AI page, "The Memory Problem": every 128 tokens
+ * collapse into a single entry.  Reading: the same per-channel softmax
+ * pooling with one series, block i = tokens m*i .. m*i+m-1:
+ *     z_s[c] = sum_e x_s[e] W[e][c] + bias[s - m*i][c]
+ *     out_i[c] = sum_s softmax_s(z_s[c]) x_s[c],   s < lens[b].
+ *   x [B][n_max][d], W [d][d] ([in][out]), bias [m][d],
+ *   out [B][ceil(n_max/m)][d]; rows i >= ceil(lens[b]/m) are set to 0.
+ * Supported: d in {32, 64, 128}; 1 <= m <= 4096.
+ * ---------------------------------------------------------------------- */
+CSA_API int hca_compress(const void *x, const int32_t *lens, int B, int n_max, int d, int m,
+                 const void *W, const void *bias, csa_dtype dt, void *out, void *stream);
+
+/* ------------------------------------------------------------------------
+ * csa_index_topk -- lightning-indexer scores and per-query top-k.
+ *
+ * Anatomy page, CSA bullet: a small lightning indexer (64 heads of 128
+ * dimensions) ranks the compressed blocks for each query, and each query
+ * attends only to the most relevant 1,024 (Flash: 512).  Exchange Rates
+ * page, section 3: ReLU-gated dot products, then top-k.  Reading:
+ *     I[t,i] = sum_h w[t,h] * max(0, q_idx[t,h,:] . k_idx[i,:])
+ * for visible entries i < floor((t+1)/4).  The selected set S_t is the k
+ * visible entries first in the order (score descending, index ascending):
+ * ties go to the lower index and -0.0 ranks as +0.0.  If fewer than k are
+ * visible, all are selected.
+ *
+ *   q_idx  [B][Tq][HI][dI]   indexer queries
+ *   w      [B][Tq][HI]       per-head indexer weights
+ *   k_idx  [B][nc_max][dI]   indexer-key cache (one key per entry)
+ *   lens, q_pos              see conventions (q_pos may be NULL)
+ *   idx_out [B][Tq][k] int32 S_t in ascending index order, padded with -1
+ *   scores_out [B][Tq][nc_max] float, optional (NULL: kept in workspace):
+ *                            I[t,i] for visible i, -inf for the rest
+ *   workspace, ws_bytes      >= csa_index_topk_workspace_size(...), 16-byte
+ *                            aligned; may be NULL when that size is 0
+ * Inputs must be finite.  Supported: (HI, dI) with HI in [1, 128] and dI in
+ * {32, 64, 128}; 1 <= k <= 4096; nc_max <= 393216 (1.5M tokens).
+ * ---------------------------------------------------------------------- */
+CSA_API size_t csa_index_topk_workspace_size(int B, int Tq, int nc_max, int has_scores_out);
+
+CSA_API int csa_index_topk(const void *q_idx, const void *w, const void *k_idx, const int32_t *lens,
+                   const int32_t *q_pos, int B, int Tq, int HI, int dI, int nc_max, int k,
+                   csa_dtype dt, int32_t *idx_out, float *scores_out, void *workspace,
+                   size_t ws_bytes, void *stream);
+
+/* ------------------------------------------------------------------------
+ * csa_index_scores / csa_topk -- the two halves of csa_index_topk, for
+ * callers that want the scores themselves or select over their own scores.
+ * csa_index_topk(...) is exactly csa_index_scores into its scores buffer
+ * followed by csa_topk on it.
+ *
+ * csa_index_scores writes scores_out [B][Tq][nc_max] (float, required):
+ * I[t,i] for visible i < floor((t+1)/4), -inf for the rest.
+ * csa_topk reads such a score array (visible entries must be finite) and
+ * writes idx_out [B][Tq][k] with the selection rule of csa_index_topk.
+ * Supported sets as for csa_index_topk.
+ * ---------------------------------------------------------------------- */
+CSA_API int csa_index_scores(const void *q_idx, const void *w, const void *k_idx,
+                             const int32_t *lens, const int32_t *q_pos, int B, int Tq, int HI,
+                             int dI, int nc_max, csa_dtype dt, float *scores_out, void *stream);
+
+CSA_API int csa_topk(const float *scores, const int32_t *lens, const int32_t *q_pos, int B, int Tq,
+                     int nc_max, int k, int32_t *idx_out, void *stream);
+
+/* ------------------------------------------------------------------------
+ * csa_attend -- sparse MQA attention over the selected entries + window.
+ *
+ * Anatomy page, "The skeleton": one key-value head is shared by every query
+ * head, and each cached entry is both the key and the value.  CSA bullet:
+ * each query attends to its selected entries.  First of the three details:
+ * every CSA layer also attends to the last 128 tokens directly.  Reading:
+ * for each head h, one joint softmax over
+ *     { kv_c[b][i] : i in idx[b][tq][:], 0 <= i < floor((t+1)/4) }
+ *   + { token s : max(0, t-window+1) <= s <= t }
+ * with logits scale * (q[t,h] . v) and output sum softmax * v.  -1 padding
+ * and indices that are not visible contribute nothing; a repeated index
+ * contributes once per occurrence.
+ *
+ *   q      [B][Tq][H][d]      queries (already normalised / rotated)
+ *   kv_c   [B][nc_max][d]     compressed KV cache
+ *   kv_tok [B][n_tok][d]      window tokens, a ring: token s at row
+ *                             s % n_tok; each query's window must fit
+ *                             (min(window, t+1) <= n_tok)
+ *   idx    [B][Tq][k] int32   selected entries (csa_index_topk output)
+ *   scale  softmax scale; <= 0 means 1/sqrt(d)
+ *   out    [B][Tq][H][d]
+ * Supported: d in {64, 128}; 1 <= H <= 128; 1 <= k <= 4096;
+ * 1 <= window <= 4096.
+ * ---------------------------------------------------------------------- */
+CSA_API int csa_attend(const void *q, const void *kv_c, const void *kv_tok, int n_tok, const int32_t *idx,
+               const int32_t *lens, const int32_t *q_pos, int B, int Tq, int H, int d, int nc_max,
+               int k, int window, float scale, csa_dtype dt, void *out, void *stream);
+
+/* ------------------------------------------------------------------------
+ * hca_attend -- dense MQA attention over every visible HCA entry + window.
+ *
+ * Anatomy page, HCA bullet: queries attend to all compressed entries
+ * densely (about 8,000 at a million tokens).  Same reading as csa_attend
+ * with the selected set replaced by every visible entry i < floor((t+1)/m).
+ *   kv_c [B][nc_max][d] HCA cache (nc_max may be 0), other arguments as for
+ *   csa_attend.  Supported: d in {64, 128}; 1 <= H <= 128; 1 <= m <= 4096;
+ *   1 <= window <= 4096; nc_max <= 65536.
+ * ---------------------------------------------------------------------- */
+CSA_API int hca_attend(const void *q, const void *kv_c, const void *kv_tok, int n_tok,
+               const int32_t *lens, const int32_t *q_pos, int B, int Tq, int H, int d, int nc_max,
+               int m, int window, float scale, csa_dtype dt, void *out, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CSA_B200_H */
