@@ -181,10 +181,16 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(const float *__restrict__
   int eq_rank = eq_before;
   for (int j = c0; j < c1; ++j) {
     const uint32_t km = keys[j] & pmask;
+    // (pos < k always holds: exactly k keys are selected; the guard keeps a
+    // miscount from ever writing outside the row)
     if (km > pval) {
-      orow[pos++] = lo + j;
+      if (pos < k) orow[pos] = lo + j;
+      ++pos;
     } else if (km == pval) {
-      if (eq_rank < take_eq) orow[pos++] = lo + j;
+      if (eq_rank < take_eq) {
+        if (pos < k) orow[pos] = lo + j;
+        ++pos;
+      }
       ++eq_rank;
     }
   }
