@@ -36,7 +36,7 @@ def build(force: bool = False, verbose: bool = False, extra_flags=()) -> str:
             and os.path.getmtime(LIB) >= max(os.path.getmtime(s) for s in srcs)):
         return LIB
     cmd = [NVCC, *NVCC_FLAGS, *extra_flags, "-I", INCLUDE, "-I", CSRC, "-shared",
-           os.path.join(CSRC, "csa_api.cu"), "-o", LIB + ".tmp", "-lcuda"]
+           os.path.join(CSRC, "csa_api.cu"), "-o", LIB + ".tmp"]
     if verbose:
         print(" ".join(cmd))
     subprocess.run(cmd, check=True)

@@ -4,11 +4,13 @@
 // The whole library is this one translation unit: every kernel header is
 // included here, so the device error word has one definition and no device
 // linking is needed.
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <algorithm>
 #include <mutex>
 #include <string>
 #include <unordered_map>
@@ -18,6 +20,7 @@
 #include "common.cuh"
 #include "compress.cuh"
 #include "index_score_fma.cuh"
+#include "index_score_tc.cuh"
 #include "topk.cuh"
 #include "attend_fma.cuh"
 
@@ -89,6 +92,58 @@ int launch_cluster(void (*kernel)(KArgs...), int cs, unsigned grid, unsigned blo
     cudaGetLastError();
     return fail(CSA_ERR_LAUNCH, "%s: launch failed: %s", what, cudaGetErrorString(e));
   }
+  return CSA_OK;
+}
+
+// Number of SMs of the current device (cached per device).
+int num_sms() {
+  static int cache[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) return 148;
+  if (cache[dev] == 0) {
+    int n = 0;
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    cache[dev] = n > 0 ? n : 148;
+  }
+  return cache[dev];
+}
+
+// cuTensorMapEncodeTiled, fetched from the driver through the runtime (no
+// link-time dependency on libcuda).
+typedef CUresult (*encode_tiled_fn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                    const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                    const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                    CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+encode_tiled_fn get_encode_tiled() {
+  static encode_tiled_fn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<encode_tiled_fn>(p);
+  });
+  return fn;
+}
+
+// 2-D bf16 tensor [outer][inner] (row-major), box [box_outer][box_inner],
+// 128-byte swizzle, zero fill outside the tensor.
+int encode_bf16_2d(CUtensorMap *map, const void *base, uint64_t inner, uint64_t outer,
+                   uint32_t box_inner, uint32_t box_outer, const char *what) {
+  encode_tiled_fn enc = get_encode_tiled();
+  if (!enc) return fail(CSA_ERR_CUDA, "%s: cuTensorMapEncodeTiled is unavailable", what);
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {inner * 2};
+  const cuuint32_t box[2] = {box_inner, box_outer};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(CSA_ERR_CUDA, "%s: tensor map encoding failed (%d)", what, (int)r);
   return CSA_OK;
 }
 
@@ -168,6 +223,49 @@ int launch_index_fma(const void *qI, const void *w, const void *kI, const int32_
                                              static_cast<const T *>(kI), lens, q_pos, Tq, HI,
                                              nc_max, scores);
   return launch_status("csa_index_topk (scores)");
+}
+
+template <int N, int DI>
+int launch_index_tc(const void *qI, const void *w, const void *kI, const int32_t *lens,
+                    const int32_t *q_pos, int R, int Tq, int HI, int nc_max, float *scores,
+                    bool fill, cudaStream_t st) {
+  const char *what = "csa_index_scores";
+  CUtensorMap tmK, tmQ;
+  const int B = R / Tq;
+  int rc = encode_bf16_2d(&tmK, kI, DI, (uint64_t)B * nc_max, 64, csa::kTcRows, what);
+  if (rc) return rc;
+  rc = encode_bf16_2d(&tmQ, qI, DI, (uint64_t)R * HI, 64, N, what);
+  if (rc) return rc;
+  constexpr size_t A_STAGE = (size_t)csa::kTcRows * DI * 2, B_SLOT = (size_t)N * DI * 2;
+  const size_t budget = 227 * 1024 - 1024 - 2 * B_SLOT - 1024;  // align slack, barriers, statics
+  const int stages = (int)std::min<size_t>(6, budget / A_STAGE);
+  const size_t smem = 1024 + stages * A_STAGE + 2 * B_SLOT + 8 * (2 * stages + 9);
+  auto kern = csa::k_index_score_tc<N, DI>;
+  rc = ensure_smem(kern, smem, what);
+  if (rc) return rc;
+  csa::IndexTcArgs a;
+  a.w = static_cast<const __nv_bfloat16 *>(w);
+  a.lens = lens;
+  a.q_pos = q_pos;
+  a.scores = scores;
+  a.Tq = Tq;
+  a.HI = HI;
+  a.nc_max = nc_max;
+  a.R = R;
+  a.stages = stages;
+  a.fill_invisible = fill ? 1 : 0;
+  kern<<<num_sms(), csa::kTcThreads, smem, st>>>(tmK, tmQ, a);
+  return launch_status(what);
+}
+
+template <int DI>
+int launch_index_tc_n(const void *qI, const void *w, const void *kI, const int32_t *lens,
+                      const int32_t *q_pos, int R, int Tq, int HI, int nc_max, float *scores,
+                      bool fill, cudaStream_t st) {
+  if (HI <= 16) return launch_index_tc<16, DI>(qI, w, kI, lens, q_pos, R, Tq, HI, nc_max, scores, fill, st);
+  if (HI <= 32) return launch_index_tc<32, DI>(qI, w, kI, lens, q_pos, R, Tq, HI, nc_max, scores, fill, st);
+  if (HI <= 64) return launch_index_tc<64, DI>(qI, w, kI, lens, q_pos, R, Tq, HI, nc_max, scores, fill, st);
+  return launch_index_tc<128, DI>(qI, w, kI, lens, q_pos, R, Tq, HI, nc_max, scores, fill, st);
 }
 
 template <int CS>
@@ -323,10 +421,17 @@ namespace {
 
 int index_scores_impl(const void *q_idx, const void *w, const void *k_idx, const int32_t *lens,
                       const int32_t *q_pos, int B, int Tq, int HI, int dI, int nc_max,
-                      csa_dtype dt, float *scores, cudaStream_t st) {
+                      csa_dtype dt, float *scores, bool fill, cudaStream_t st) {
   const int R = B * Tq;
   if (R == 0 || nc_max == 0) return CSA_OK;
   if (R > 65535) return fail(CSA_ERR_UNSUPPORTED, "csa_index_scores: B*Tq=%d > 65535", R);
+  // bf16 with 128-byte key rows or wider: the tensor-core kernel
+  if (dt == CSA_BF16 && (dI == 64 || dI == 128)) {
+    if ((long)B * nc_max >= (1L << 31) || (long)R * HI >= (1L << 31))
+      return fail(CSA_ERR_UNSUPPORTED, "csa_index_scores: tensor too large for 32-bit coordinates");
+    return dI == 64 ? launch_index_tc_n<64>(q_idx, w, k_idx, lens, q_pos, R, Tq, HI, nc_max, scores, fill, st)
+                    : launch_index_tc_n<128>(q_idx, w, k_idx, lens, q_pos, R, Tq, HI, nc_max, scores, fill, st);
+  }
   if (dt == CSA_F32) {
     switch (dI) {
       case 32: return launch_index_fma<float, 32>(q_idx, w, k_idx, lens, q_pos, R, Tq, HI, nc_max, scores, st);
@@ -391,7 +496,7 @@ int csa_index_scores(const void *q_idx, const void *w, const void *k_idx, const 
   if (!aligned16(q_idx) || !aligned16(w) || !aligned16(k_idx) || !aligned16(scores_out))
     return fail(CSA_ERR_ALIGN, "%s: tensors must be 16-byte aligned", what);
   return index_scores_impl(q_idx, w, k_idx, lens, q_pos, B, Tq, HI, dI, nc_max, dt, scores_out,
-                           static_cast<cudaStream_t>(stream));
+                           true, static_cast<cudaStream_t>(stream));
 }
 
 int csa_topk(const float *scores, const int32_t *lens, const int32_t *q_pos, int B, int Tq,
@@ -427,7 +532,8 @@ int csa_index_topk(const void *q_idx, const void *w, const void *k_idx, const in
   if (need > 0 && !aligned16(workspace)) return fail(CSA_ERR_ALIGN, "%s: workspace must be 16-byte aligned", what);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   float *scores = scores_out ? scores_out : static_cast<float *>(workspace);
-  rc = index_scores_impl(q_idx, w, k_idx, lens, q_pos, B, Tq, HI, dI, nc_max, dt, scores, st);
+  rc = index_scores_impl(q_idx, w, k_idx, lens, q_pos, B, Tq, HI, dI, nc_max, dt, scores,
+                         scores_out != nullptr, st);
   if (rc) return rc;
   return topk_impl(scores, lens, q_pos, B, Tq, nc_max, k, idx_out, st);
 }

@@ -18,6 +18,10 @@ except Exception:  # pragma: no cover
 F32_ATOL = 1e-5
 BF16_ATOL, BF16_RTOL = 2e-2, 1e-2
 SCORE_EPS = {"f32": 1e-5, "bf16": 1e-3}
+# Scores computed from caches that the GPU chain built itself: each bf16 cache
+# element may sit one bf16 ulp (2^-8 relative) away from the oracle's rounding
+# of the exact value, so the end-to-end score bound is the looser 1e-2 (1+|s|).
+CHAIN_EPS = {"f32": 1e-5, "bf16": 1e-2}
 
 
 def to_dev(a, device="cuda"):
@@ -55,8 +59,8 @@ def assert_close(got, ref64, dt, what=""):
                                f"worst {np.abs(g - ref64).max():.3g}")
 
 
-def assert_scores_close(gpu_scores, ref64, vis, dt, what="scores"):
-    eps = SCORE_EPS[dt]
+def assert_scores_close(gpu_scores, ref64, vis, dt, what="scores", eps=None):
+    eps = SCORE_EPS[dt] if eps is None else eps
     for r in range(ref64.shape[0]):
         v = int(vis[r])
         g = gpu_scores[r, :v].astype(np.float64)
@@ -66,11 +70,11 @@ def assert_scores_close(gpu_scores, ref64, vis, dt, what="scores"):
         assert np.all(np.isneginf(gpu_scores[r, v:])), f"{what} row {r}: invisible entries not -inf"
 
 
-def topk_set_difference_ok(gpu_idx, ref_idx, ref_scores, k, dt):
+def topk_set_difference_ok(gpu_idx, ref_idx, ref_scores, k, dt, eps=None):
     """Level (ii): the GPU and oracle index sets may differ only in entries
     whose oracle score lies within eps of the oracle's k-th score.  Returns
     the number of differing entries (asserts the rest)."""
-    eps = SCORE_EPS[dt]
+    eps = SCORE_EPS[dt] if eps is None else eps
     diff = 0
     for r in range(gpu_idx.shape[0]):
         a = set(int(i) for i in gpu_idx[r] if i >= 0)

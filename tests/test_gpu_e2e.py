@@ -12,7 +12,7 @@ import pytest
 
 import oracle
 import workloads as W
-from tests.helpers import (assert_close, assert_scores_close, to_dev, to_host,
+from tests.helpers import (CHAIN_EPS, assert_close, assert_scores_close, to_dev, to_host,
                            topk_set_difference_ok)
 
 pytestmark = pytest.mark.gpu
@@ -74,8 +74,15 @@ def test_workload2_csa_prefill_sampled_rows():
     sub = lambda a: a[:, rows]
     ref_idx, ref_sc = oracle.index_topk(sub(wl["qI"]), sub(wl["w"]), KI_r, wl["lens"], k, q_pos)
     vis = oracle.visible(wl["lens"], 1, len(rows), 4, q_pos).reshape(-1)
-    assert_scores_close(sc[0, rows], ref_sc[0], vis, "bf16")
-    topk_set_difference_ok(idx[0, rows], ref_idx[0], ref_sc[0], k, "bf16")
+    # the chain: scores from the GPU-built cache (bound CHAIN_EPS), the
+    # selection bit-exact on the GPU's own scores
+    assert_scores_close(sc[0, rows], ref_sc[0], vis, "bf16", eps=CHAIN_EPS["bf16"])
+    np.testing.assert_array_equal(idx[0, rows], oracle.select_topk(sc[0, rows], vis, k))
+    topk_set_difference_ok(idx[0, rows], ref_idx[0], ref_sc[0], k, "bf16", eps=CHAIN_EPS["bf16"])
+    # stage-wise: the GPU indexer on the oracle's cache, at the tight bound
+    sc2 = to_host(csa.csa_index_scores(to_dev(sub(wl["qI"])), to_dev(sub(wl["w"])), to_dev(KI_r),
+                                       D["lens"], q_pos=to_dev(q_pos)))
+    assert_scores_close(sc2[0], ref_sc[0], vis, "bf16")
     ref_out = oracle.attend(sub(wl["q"]), C_r, wl["x"], wl["lens"], idx=ref_idx, q_pos=q_pos, window=window)
     for j, r in enumerate(rows):
         if set(idx[0, r]) == set(ref_idx[0, j]):

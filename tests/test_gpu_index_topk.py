@@ -71,6 +71,21 @@ def test_bf16_tiles_and_cluster_sizes(nc):
     check_all(qI, w, kI, lens, 1024, "bf16")
 
 
+@pytest.mark.parametrize("HI,dI", [(4, 128), (16, 64), (24, 128), (100, 64), (128, 128), (64, 32)])
+def test_bf16_head_and_dim_shapes(HI, dI):
+    """Indexer head counts that pad to 16/32/128 tensor-core columns, key
+    widths of one and two 128-byte slices, and the 32-wide keys that take the
+    CUDA-core kernel; several query rows per sequence at explicit positions."""
+    seed = 1000 + HI + dI
+    B, Tq, nc = 2, 3, 1000
+    lens = np.array([4 * nc, 4 * nc - 333], np.int32)
+    q_pos = np.array([[3999, 2500, 130], [3666, 515, 1]], np.int32)
+    qI = W.normal(seed, "qI", (B, Tq, HI, dI), 1.0, "bf16")
+    w = W.normal(seed, "w", (B, Tq, HI), 1.0 / HI, "bf16")
+    kI = W.normal(seed, "kI", (B, nc, dI), 1.0, "bf16")
+    check_all(qI, w, kI, lens, 200, "bf16", q_pos=q_pos)
+
+
 def test_causal_rows_prefill_like():
     """Many query rows at increasing positions (v from 0 to > k): visibility
     and the v <= k / v == 0 paths."""
@@ -103,7 +118,7 @@ def test_exact_zero_ties_straddle_threshold():
     exactly 0 (every head's ReLU is 0); with positive head weights the rest
     score > 0, and k larger than the positive set forces the tie rule onto
     the zeros."""
-    nc, k = 9000, 6000
+    nc, k = 6000, 4000
     g = np.random.default_rng(12)
     q = np.abs(g.standard_normal((1, 1, 64, 128))).astype(np.float32)
     keys = np.abs(g.standard_normal((1, nc, 128))).astype(np.float32)
