@@ -82,6 +82,20 @@ def scoring_kernel_bytes(s, B):
 # --------------------------------------------------------------------------
 # clocks during the timed region
 # --------------------------------------------------------------------------
+def smi_index(uuid, fallback):
+    """nvidia-smi's index of the GPU with this UUID (CUDA may renumber)."""
+    try:
+        out = subprocess.run(["nvidia-smi", "--query-gpu=index,uuid", "--format=csv,noheader"],
+                             capture_output=True, text=True, timeout=20).stdout
+        for ln in out.splitlines():
+            idx, u = [x.strip() for x in ln.split(",")[:2]]
+            if uuid.replace("GPU-", "") in u:
+                return idx
+    except Exception:
+        pass
+    return str(fallback)
+
+
 class ClockSampler:
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -182,7 +196,7 @@ def run_ours(args, rank, world, dev):
     K = args.steps
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    sampler = ClockSampler(f"GPU-{torch.cuda.get_device_properties(dev).uuid}")
+    sampler = ClockSampler(smi_index(str(torch.cuda.get_device_properties(dev).uuid), dev))
     if rank == 0:
         sampler.start()
     barrier()
