@@ -1,0 +1,283 @@
+// attend_tc.cuh -- single-KV-head attention over selected (CSA) or all (HCA)
+// compressed entries plus the sliding window, on the tcgen05 tensor cores.
+// bf16 inputs, head dim 128, up to 128 query heads.
+//
+// "Anatomy of a Frontier Model: Reading DeepSeek-V4 Through Part V":
+// "The skeleton, and what's kept" (one key-value head shared by all query
+// heads; the cached entry is both key and value), CSA and HCA bullets (the
+// selected / all entries), first of the "three details" (every layer also
+// attends to the last 128 tokens under the same softmax).
+//
+// One query row per cluster of CS CTAs; CTA `rank` takes a contiguous range
+// of the row's key list ([selected entries] ++ [window tokens]) in tiles of
+// up to 256 keys.  Per tile:
+//   gather  cp.async 16-byte chunks of the key rows into shared memory in the
+//           128-byte-swizzled layout (invalid slots are zero-filled);
+//   S = Q K^T   tcgen05.mma, M = 128 (heads, zero-padded), N = tile keys,
+//           K = 128; A = Q (K-major), B = the key tile (K-major);
+//   softmax thread h owns TMEM lane h = head h: base-2 online softmax over
+//           its row of S; P (bf16) written back in the swizzled K-major layout;
+//   O = P V  tcgen05.mma, M = 128, N = 128 (head dim), K = tile keys;
+//           A = P, B = the SAME key tile read MN-major (the entry is the value);
+//   accumulate  O is read back per lane and folded into registers with the
+//           running rescale.
+// The CTAs' partial (max, sum, output) merge through distributed shared
+// memory in fixed rank order, as in the CUDA-core kernel.
+#pragma once
+
+#include <cooperative_groups.h>
+
+#include "attend_fma.cuh"
+#include "common.cuh"
+#include "sm100.cuh"
+
+namespace csa {
+
+constexpr int kAtThreads = 128;
+constexpr int kAtMaxTile = 256;                      // keys per tile
+constexpr uint32_t kAtQAtom = 128 * 128;             // 128 rows x 128 B
+constexpr uint32_t kAtKHalf = kAtMaxTile * 128;      // one 64-wide d slice of the key tile
+constexpr uint32_t kAtPAtom = 128 * 128;             // 128 heads x 64 keys x 2 B
+constexpr size_t kAtSmem = 1024 + 2 * kAtQAtom + 2 * kAtKHalf + 4 * kAtPAtom;
+
+template <int CS>
+__global__ void __launch_bounds__(kAtThreads, 1) k_attend_tc(AttendArgs a) {
+  using namespace sm100;
+  constexpr int D = 128;
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ uint32_t tmem_holder;
+  __shared__ uint64_t bar_s, bar_o;
+  __shared__ int kvalid[kAtMaxTile];
+  __shared__ float pm[128], pl[128];
+  __shared__ int abort_flag;
+
+  uint8_t *base = reinterpret_cast<uint8_t *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t *sQ = base;
+  uint8_t *sK = sQ + 2 * kAtQAtom;
+  uint8_t *sP = sK + 2 * kAtKHalf;
+  float *part = reinterpret_cast<float *>(base);  // [128][128] partial outputs, after the loop
+
+  const int rank = (CS > 1) ? (int)cg::this_cluster().block_rank() : 0;
+  const int r = blockIdx.x / CS;
+  const int b = r / a.Tq, tq = r % a.Tq;
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const int H = a.H;
+  const __nv_bfloat16 *q = static_cast<const __nv_bfloat16 *>(a.q);
+  const __nv_bfloat16 *kv_c = static_cast<const __nv_bfloat16 *>(a.kv_c);
+  const __nv_bfloat16 *kv_tok = static_cast<const __nv_bfloat16 *>(a.kv_tok);
+  __nv_bfloat16 *out = static_cast<__nv_bfloat16 *>(a.out) + (size_t)r * H * D;
+
+  int t;
+  bool ok = query_position(a.lens, a.q_pos, b, a.Tq, tq, t);
+  int v = 0, w0 = 0, nwin = 0;
+  if (ok) {
+    v = (t + 1) / a.m;
+    w0 = max(0, t - a.window + 1);
+    nwin = t - w0 + 1;
+    if (v > a.nc_max) {
+      if (tid == 0 && rank == 0) raise_dev_err(kDevErrCache);
+      ok = false;
+    } else if (nwin > a.n_tok) {
+      if (tid == 0 && rank == 0) raise_dev_err(kDevErrRing);
+      ok = false;
+    }
+  }
+  if (!ok) {  // uniform over the cluster
+    for (int u = tid; u < H * D; u += kAtThreads)
+      if ((u / D) % CS == rank) out[u] = __float2bfloat16_rn(0.f);
+    return;
+  }
+
+  const int nsel = a.idx ? a.k : v;
+  const int L = nsel + nwin;
+  const int per = (L + CS - 1) / CS;
+  const int lo = min(L, rank * per), hi = min(L, lo + per);
+
+  if (warp == 0) {
+    tmem_alloc(smem_u32(&tmem_holder), 512);
+    tmem_relinquish();
+  }
+  if (tid == 0) {
+    abort_flag = 0;
+    mbar_init(smem_u32(&bar_s), 1);
+    mbar_init(smem_u32(&bar_o), 1);
+    fence_barrier_init();
+  }
+  // Q rows (heads) in the swizzled K-major layout; heads >= H are zero rows
+  const __nv_bfloat16 *qrow = q + (size_t)r * H * D;
+  for (int u = tid; u < 128 * 16; u += kAtThreads) {
+    const int h = u >> 4, c = u & 15;
+    const uint32_t dst = smem_u32(sQ) + (c >> 3) * kAtQAtom + h * 128 + (((c & 7) ^ (h & 7)) << 4);
+    cp_async16(dst, h < H ? qrow + (size_t)h * D + c * 8 : qrow, h < H ? 16u : 0u);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tS = tmem_holder, tO = tmem_holder + 256;
+  const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+  volatile int *abort = &abort_flag;
+
+  float o[D];
+#pragma unroll
+  for (int e = 0; e < D; ++e) o[e] = 0.f;
+  float m_run = -INFINITY, l_run = 0.f;
+  uint32_t ns = 0, no = 0;
+  bool alive = true;
+
+  for (int p0 = lo; p0 < hi && alive; p0 += kAtMaxTile) {
+    const int ntile = min(kAtMaxTile, hi - p0);
+    const int nchunk = (ntile + 31) >> 5;  // 32-key chunks; MMA N = 32 * nchunk
+    // ---- gather the key rows (16 chunks of 16 B each)
+    for (int u = tid; u < nchunk * 32 * 16; u += kAtThreads) {
+      const int j = u >> 4, c = u & 15;
+      const int p = p0 + j;
+      const __nv_bfloat16 *row = nullptr;
+      if (j < ntile) {
+        if (p < nsel) {
+          const int i = a.idx ? __ldg(a.idx + (size_t)r * a.k + p) : p;
+          if (i >= 0 && i < v) row = kv_c + ((size_t)b * a.nc_max + i) * D;
+        } else {
+          const int s = w0 + (p - nsel);
+          row = kv_tok + ((size_t)b * a.n_tok + (s % a.n_tok)) * D;
+        }
+      }
+      if (c == 0) kvalid[j] = row != nullptr;
+      const uint32_t dst = smem_u32(sK) + (c >> 3) * kAtKHalf + j * 128 + (((c & 7) ^ (j & 7)) << 4);
+      cp_async16(dst, row ? row + c * 8 : kv_tok, row ? 16u : 0u);
+    }
+    cp_async_wait_all();
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    // ---- S = Q K^T
+    if (tid == 0) {
+      const uint32_t idesc = idesc_bf16_f32(128, 32 * nchunk);
+#pragma unroll
+      for (int k = 0; k < D / 16; ++k) {
+        const uint32_t off = (k >> 2) * kAtQAtom + (k & 3) * 32;
+        const uint32_t koff = (k >> 2) * kAtKHalf + (k & 3) * 32;
+        umma_bf16(tS, sdesc_kmajor_sw128(smem_u32(sQ) + off), sdesc_kmajor_sw128(smem_u32(sK) + koff),
+                  idesc, k > 0);
+      }
+      umma_commit(smem_u32(&bar_s));
+    }
+    alive = mbar_wait(smem_u32(&bar_s), ns & 1, abort);
+    alive = __syncthreads_and(alive);
+    ++ns;
+    if (!alive) break;
+    tc_fence_after();
+    // ---- softmax over this lane's (head's) row
+    float mt = -INFINITY;
+    for (int c = 0; c < nchunk; ++c) {
+      uint32_t sv[32];
+      tmem_ld16(tS + lane_off + 32 * c, sv);
+      tmem_ld16(tS + lane_off + 32 * c + 16, sv + 16);
+      tmem_wait_ld_regs<32>(sv);
+#pragma unroll
+      for (int jj = 0; jj < 32; ++jj)
+        if (kvalid[32 * c + jj]) mt = fmaxf(mt, __uint_as_float(sv[jj]) * a.scale_log2);
+    }
+    const float m_new = fmaxf(m_run, mt);
+    const float alpha = (m_new == -INFINITY) ? 1.f : exp2f(m_run - m_new);
+    float lsum = 0.f;
+    for (int c = 0; c < nchunk; ++c) {
+      uint32_t sv[32];
+      tmem_ld16(tS + lane_off + 32 * c, sv);
+      tmem_ld16(tS + lane_off + 32 * c + 16, sv + 16);
+      tmem_wait_ld_regs<32>(sv);
+#pragma unroll
+      for (int g = 0; g < 4; ++g) {  // 8 keys -> one 16-byte chunk of P
+        uint32_t pk[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int j0 = 8 * g + 2 * e;
+          const float p0v = kvalid[32 * c + j0] ? exp2f(__uint_as_float(sv[j0]) * a.scale_log2 - m_new) : 0.f;
+          const float p1v = kvalid[32 * c + j0 + 1] ? exp2f(__uint_as_float(sv[j0 + 1]) * a.scale_log2 - m_new) : 0.f;
+          lsum += p0v + p1v;
+          __nv_bfloat162 pr = __floats2bfloat162_rn(p0v, p1v);
+          pk[e] = *reinterpret_cast<uint32_t *>(&pr);
+        }
+        const int kg = 4 * c + g;  // 8-key group index 0..31
+        const uint32_t dst = smem_u32(sP) + (kg >> 3) * kAtPAtom + tid * 128 + (((kg & 7) ^ (tid & 7)) << 4);
+        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(pk[0]), "r"(pk[1]),
+                     "r"(pk[2]), "r"(pk[3])
+                     : "memory");
+      }
+    }
+    if (m_new != -INFINITY) {
+      l_run = l_run * alpha + lsum;
+      m_run = m_new;
+    }
+    tc_fence_before();
+    fence_proxy_async_smem();
+    __syncthreads();
+    tc_fence_after();
+    // ---- O = P V (the key tile read MN-major as the value operand)
+    if (tid == 0) {
+      const uint32_t idesc = idesc_bf16_f32_bmn(128, D);
+      for (int k = 0; k < 2 * nchunk; ++k) {  // 16 keys per MMA
+        const uint32_t poff = (k >> 2) * kAtPAtom + (k & 3) * 32;
+        umma_bf16(tO, sdesc_kmajor_sw128(smem_u32(sP) + poff),
+                  sdesc_mnmajor_sw128(smem_u32(sK) + k * 2048, kAtKHalf), idesc, k > 0);
+      }
+      umma_commit(smem_u32(&bar_o));
+    }
+    alive = mbar_wait(smem_u32(&bar_o), no & 1, abort);
+    alive = __syncthreads_and(alive);
+    ++no;
+    if (!alive) break;
+    tc_fence_after();
+    const float scl = (m_new == -INFINITY) ? 1.f : alpha;
+#pragma unroll
+    for (int c = 0; c < D / 32; ++c) {
+      uint32_t ov[32];
+      tmem_ld16(tO + lane_off + 32 * c, ov);
+      tmem_ld16(tO + lane_off + 32 * c + 16, ov + 16);
+      tmem_wait_ld_regs<32>(ov);
+#pragma unroll
+      for (int jj = 0; jj < 32; ++jj) o[32 * c + jj] = fmaf(o[32 * c + jj], scl, __uint_as_float(ov[jj]));
+    }
+    tc_fence_before();
+    __syncthreads();  // every lane done with S, P and O before they are rewritten
+  }
+
+  // ---- publish partials (rotated columns: conflict-free rows in shared memory)
+  __syncthreads();
+  if (tid < H) {
+    pm[tid] = m_run;
+    pl[tid] = l_run;
+#pragma unroll
+    for (int e = 0; e < D; ++e) part[tid * D + ((e + tid) & (D - 1))] = o[e];
+  }
+  att_cluster_sync<CS>();
+  const int nmine = (H - rank + CS - 1) / CS;
+  for (int u = tid; u < nmine * D; u += kAtThreads) {
+    const int h = rank + CS * (u / D), e = u % D;
+    float M = -INFINITY;
+#pragma unroll
+    for (int c = 0; c < CS; ++c) M = fmaxf(M, att_peer<CS>(pm, c)[h]);
+    float Ls = 0.f, Os = 0.f;
+#pragma unroll
+    for (int c = 0; c < CS; ++c) {
+      const float mc = att_peer<CS>(pm, c)[h];
+      if (mc == -INFINITY) continue;
+      const float wgt = exp2f(mc - M);
+      Ls = fmaf(att_peer<CS>(pl, c)[h], wgt, Ls);
+      Os = fmaf(att_peer<CS>(part, c)[h * D + ((e + h) & (D - 1))], wgt, Os);
+    }
+    out[(size_t)h * D + e] = __float2bfloat16_rn(Os / Ls);
+  }
+  att_cluster_sync<CS>();
+  if (tid == 0 && abort_flag) raise_dev_err(kDevErrTimeout);
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem_holder, 512);
+  }
+}
+
+}  // namespace csa

@@ -20,6 +20,7 @@ enum DevErr : int {
   kDevErrLen = 2,    // lens[b] < 0 or > n_max
   kDevErrCache = 3,  // visible entries exceed the cache rows
   kDevErrRing = 4,   // a query's window does not fit the token ring
+  kDevErrTimeout = 5,  // a tensor-core pipeline wait passed its time limit
 };
 
 __device__ int g_dev_err;

@@ -23,6 +23,7 @@
 #include "index_score_tc.cuh"
 #include "topk.cuh"
 #include "attend_fma.cuh"
+#include "attend_tc.cuh"
 
 namespace {
 
@@ -301,6 +302,24 @@ int launch_attend_fma(const csa::AttendArgs &a, int R, long max_keys, cudaStream
   return launch_cluster(kern, cs, (unsigned)cs * R, csa::kAttThreads, smem, st, what, a);
 }
 
+// Tensor-core attention (bf16, d = 128): enough clusters to fill the GPU
+// when the batch is small, one CTA per row when rows alone fill it.
+int launch_attend_tc(const csa::AttendArgs &a, int R, cudaStream_t st, const char *what) {
+  const int want = (2 * num_sms() + R - 1) / R;
+  int cs = 1;
+  while (cs < 8 && cs < want) cs *= 2;
+  void (*kern)(csa::AttendArgs) = nullptr;
+  switch (cs) {
+    case 1: kern = csa::k_attend_tc<1>; break;
+    case 2: kern = csa::k_attend_tc<2>; break;
+    case 4: kern = csa::k_attend_tc<4>; break;
+    default: kern = csa::k_attend_tc<8>; break;
+  }
+  int rc = ensure_smem(kern, csa::kAtSmem, what);
+  if (rc) return rc;
+  return launch_cluster(kern, cs, (unsigned)cs * R, csa::kAtThreads, csa::kAtSmem, st, what, a);
+}
+
 int attend_common(const void *q, const void *kv_c, const void *kv_tok, int n_tok,
                   const int32_t *idx, const int32_t *lens, const int32_t *q_pos, int B, int Tq,
                   int H, int d, int nc_max, int k, int m, int window, float scale, csa_dtype dt,
@@ -343,8 +362,8 @@ int attend_common(const void *q, const void *kv_c, const void *kv_tok, int n_tok
   if (dt == CSA_F32)
     return d == 64 ? launch_attend_fma<float, 64>(a, R, max_keys, st, what)
                    : launch_attend_fma<float, 128>(a, R, max_keys, st, what);
-  return d == 64 ? launch_attend_fma<__nv_bfloat16, 64>(a, R, max_keys, st, what)
-                 : launch_attend_fma<__nv_bfloat16, 128>(a, R, max_keys, st, what);
+  if (d == 128) return launch_attend_tc(a, R, st, what);
+  return launch_attend_fma<__nv_bfloat16, 64>(a, R, max_keys, st, what);
 }
 
 }  // namespace

@@ -35,7 +35,6 @@ namespace csa {
 
 constexpr int kTcRows = 128;      // entries per tile = MMA M
 constexpr int kTcThreads = 192;   // producer, MMA, 4 epilogue warps
-constexpr int kDevErrTimeout = 5; // a pipeline wait passed its time limit
 
 struct IndexTcArgs {
   const __nv_bfloat16 *w;  // [R][HI]
