@@ -49,6 +49,7 @@ __global__ void __launch_bounds__(kAtThreads, 1) k_attend_tc(AttendArgs a) {
   __shared__ uint64_t bar_s, bar_o;
   __shared__ int kvalid[kAtMaxTile];
   __shared__ float pm[128], pl[128];
+  __shared__ float mw[136], minv[128];  // merge weights [head][rank], 1 / sum
   __shared__ int abort_flag;
 
   uint8_t *base = reinterpret_cast<uint8_t *>(
@@ -243,31 +244,57 @@ __global__ void __launch_bounds__(kAtThreads, 1) k_attend_tc(AttendArgs a) {
     __syncthreads();  // every lane done with S, P and O before they are rewritten
   }
 
-  // ---- publish partials (rotated columns: conflict-free rows in shared memory)
+  // ---- publish partials: row h of `part` holds head h's output as 32
+  // float4 slots rotated by h (conflict-free stores, float4 peer reads)
   __syncthreads();
   if (tid < H) {
     pm[tid] = m_run;
     pl[tid] = l_run;
+    float4 *prow = reinterpret_cast<float4 *>(part + (size_t)tid * D);
 #pragma unroll
-    for (int e = 0; e < D; ++e) part[tid * D + ((e + tid) & (D - 1))] = o[e];
+    for (int j = 0; j < D / 4; ++j)
+      prow[(j + tid) & (D / 4 - 1)] = make_float4(o[4 * j], o[4 * j + 1], o[4 * j + 2], o[4 * j + 3]);
   }
   att_cluster_sync<CS>();
+  // merge weights of this CTA's heads (h = rank + CS * hl), ranks in order
   const int nmine = (H - rank + CS - 1) / CS;
-  for (int u = tid; u < nmine * D; u += kAtThreads) {
-    const int h = rank + CS * (u / D), e = u % D;
+  if (tid < nmine) {
+    const int h = rank + CS * tid;
     float M = -INFINITY;
 #pragma unroll
     for (int c = 0; c < CS; ++c) M = fmaxf(M, att_peer<CS>(pm, c)[h]);
-    float Ls = 0.f, Os = 0.f;
+    float Ls = 0.f;
 #pragma unroll
     for (int c = 0; c < CS; ++c) {
       const float mc = att_peer<CS>(pm, c)[h];
-      if (mc == -INFINITY) continue;
-      const float wgt = exp2f(mc - M);
+      const float wgt = (mc == -INFINITY) ? 0.f : exp2f(mc - M);
       Ls = fmaf(att_peer<CS>(pl, c)[h], wgt, Ls);
-      Os = fmaf(att_peer<CS>(part, c)[h * D + ((e + h) & (D - 1))], wgt, Os);
+      mw[tid * CS + c] = wgt;
     }
-    out[(size_t)h * D + e] = __float2bfloat16_rn(Os / Ls);
+    minv[tid] = 1.f / Ls;
+  }
+  __syncthreads();
+  for (int u = tid; u < nmine * (D / 4); u += kAtThreads) {
+    const int hl = u / (D / 4), j = u % (D / 4);
+    const int h = rank + CS * hl;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int c = 0; c < CS; ++c) {
+      const float wgt = mw[hl * CS + c];
+      if (wgt == 0.f) continue;
+      const float4 p = reinterpret_cast<const float4 *>(att_peer<CS>(part, c) + (size_t)h * D)[(j + h) & (D / 4 - 1)];
+      acc.x = fmaf(p.x, wgt, acc.x);
+      acc.y = fmaf(p.y, wgt, acc.y);
+      acc.z = fmaf(p.z, wgt, acc.z);
+      acc.w = fmaf(p.w, wgt, acc.w);
+    }
+    const float il = minv[hl];
+    __nv_bfloat162 lo2 = __floats2bfloat162_rn(acc.x * il, acc.y * il);
+    __nv_bfloat162 hi2 = __floats2bfloat162_rn(acc.z * il, acc.w * il);
+    uint2 pk;
+    pk.x = *reinterpret_cast<uint32_t *>(&lo2);
+    pk.y = *reinterpret_cast<uint32_t *>(&hi2);
+    *reinterpret_cast<uint2 *>(out + (size_t)h * D + 4 * j) = pk;
   }
   att_cluster_sync<CS>();
   if (tid == 0 && abort_flag) raise_dev_err(kDevErrTimeout);

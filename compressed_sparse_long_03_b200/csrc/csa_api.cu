@@ -153,7 +153,7 @@ int check_dtype(csa_dtype dt, const char *what) {
   return CSA_OK;
 }
 
-constexpr int kMaxIndexEntries = csa::kTopkMaxCluster * csa::kTopkSliceCap;  // 393216
+constexpr int kMaxIndexEntries = csa::kTopkMaxCluster * csa::kTopkSliceCap;  // 327680
 
 int topk_cluster_size(int nc_max) {
   int cs = 1;
@@ -273,7 +273,7 @@ template <int CS>
 int launch_topk(const float *scores, const int32_t *lens, const int32_t *q_pos, int R, int Tq,
                 int nc_max, int k, int32_t *idx_out, cudaStream_t st) {
   const int per = (nc_max + CS - 1) / CS;
-  const size_t smem = sizeof(uint32_t) * (size_t)(per > 0 ? per : 1);
+  const size_t smem = csa::topk_dyn_bytes(per > 0 ? per : 1);
   auto kern = csa::k_topk<CS>;
   int rc = ensure_smem(kern, smem, "csa_index_topk");
   if (rc) return rc;

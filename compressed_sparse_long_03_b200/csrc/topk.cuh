@@ -1,28 +1,32 @@
-// topk.cuh -- per-query top-k over indexer scores: radix select across a
+// topk.cuh -- per-query top-k over indexer scores, one query row per
 // thread-block cluster, output in ascending index order.
 //
 // "Anatomy of a Frontier Model: Reading DeepSeek-V4 Through Part V", CSA
 // bullet: each query attends to only its k most relevant entries (1,024 in
 // Pro, 512 in Flash).  The selected set is the k visible entries first in
 // the order (score desc, index asc): ties go to the lower index; -0.0 ranks
-// as +0.0; all visible entries when fewer than k.
+// as +0.0; every visible entry when fewer than k.
 //
-// Design (one query row per cluster of CS CTAs, no global scratch, no spin
-// waits):
-//  1. each CTA loads its contiguous slice of the visible scores into shared
-//     memory as order-preserving u32 keys (larger key = larger score);
-//  2. four MSB-first 8-bit radix passes find the k-th largest key T: each CTA
-//     histograms its slice (keys matching the prefix found so far), the
-//     cluster barrier publishes the histograms, and every CTA sums all CS of
-//     them through distributed shared memory in the same fixed order, so all
-//     agree on the next digit without another exchange; a pass stops early
-//     when the chosen bin holds exactly the keys still needed;
-//  3. selection is then exact: keys above the threshold prefix are in; of
-//     the keys equal to it, the lowest-index ones fill the rest.  Per-CTA
-//     counts are exchanged once more and each CTA writes its selected indices
-//     at fixed offsets, which yields the ascending-index output directly.
-// Everything is integer work, so the result is bit-exact and independent of
-// launch configuration.
+// Design (cluster of CS CTAs per row; no global scratch; no spin waits):
+//  A. each CTA loads a contiguous slice of the row's visible scores into
+//     shared memory as order-preserving u32 keys and reduces their min/max;
+//     the cluster agrees on the row's [min, max];
+//  B. a 2048-bin histogram whose bins split [min, max] evenly by value.  The
+//     bin function is monotone in the score (round-to-nearest subtract and
+//     multiply are monotone), so bins order keys exactly: the bin b* holding
+//     the k-th largest key, and the count above it, decide every key outside
+//     b*.  Bins by value (not by leading bits) keep the shared-memory atomics
+//     free of hot spots, because fp32 scores share their leading bits;
+//  C. the few keys inside b* ("candidates") are ranked exactly: every CTA
+//     reads all candidates of the cluster through distributed shared memory
+//     and counts, for each of its own, the candidates that beat it under
+//     (score desc, index asc).  When b* holds too many keys for that (a
+//     degenerate distribution, e.g. all scores equal), an MSB-first 8-bit
+//     radix select over the keys of b* takes over;
+//  D. per-CTA counts of selected keys give each CTA its output offset, and
+//     each CTA writes its selected indices in order.
+// All decisions are integer comparisons on the same keys in every CTA, so
+// the result is bit-exact and independent of the launch configuration.
 #pragma once
 
 #include <cooperative_groups.h>
@@ -34,15 +38,28 @@ namespace csa {
 namespace cg = cooperative_groups;
 
 constexpr int kTopkThreads = 512;
-constexpr int kTopkSliceCap = 49152;  // keys per CTA held in shared memory
+constexpr int kTopkSliceCap = 40960;  // keys per CTA held in shared memory
 constexpr int kTopkMaxCluster = 8;
+constexpr int kTopkBins = 2048;
+constexpr int kTopkRankCap = 512;     // candidates of a row ranked directly
 
 struct TopkShared {
-  int hist[2][256];
+  int hist[kTopkBins];
   int scan[33];
-  int digit_info[4];   // [0] chosen bin, [1] keys above it, [2] keys in it
-  int cta_counts[2];   // this CTA's (greater, equal) counts, read by peers
+  uint32_t red[2][kTopkThreads / 32];  // per-warp min / max
+  uint32_t kmin, kmax;                 // this CTA's min / max key
+  int info[4];                         // [0] bin, [1] count above it, [2] count in it
+  int ncand;                           // this CTA's candidates (keys in b*)
+  int cta_counts[2];                   // this CTA's (selected, tied) counts
+  uint32_t all_key[kTopkRankCap];
+  int all_idx[kTopkRankCap];
 };
+
+// Dynamic shared memory of one CTA for slices of up to `per` keys: the keys,
+// the candidate positions and the selection bit mask.
+__host__ __device__ constexpr size_t topk_dyn_bytes(int per) {
+  return 4ull * ((size_t)per + (size_t)(per < kTopkRankCap ? per : kTopkRankCap) + ((size_t)per + 31) / 32);
+}
 
 template <int CS>
 __device__ __forceinline__ void cluster_barrier() {
@@ -53,13 +70,26 @@ __device__ __forceinline__ void cluster_barrier() {
   }
 }
 
-template <int CS>
-__device__ __forceinline__ const TopkShared *peer(TopkShared *mine, int rank) {
+template <int CS, typename P>
+__device__ __forceinline__ P *peer_ptr(P *mine, int rank) {
   if constexpr (CS > 1) {
     return cg::this_cluster().map_shared_rank(mine, rank);
   } else {
     return mine;
   }
+}
+
+__device__ __forceinline__ float key_to_float(uint32_t k) {
+  const uint32_t u = (k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k;
+  return __uint_as_float(u);
+}
+
+// Monotone value bin of a key in [fmin, fmax] (scale = bins / (fmax - fmin);
+// scale == 0 puts every key in bin 0).
+__device__ __forceinline__ int value_bin(uint32_t key, float fmin, float scale) {
+  const float x = __fmul_rn(__fsub_rn(key_to_float(key), fmin), scale);
+  const int b = (int)x;  // x >= 0
+  return b < kTopkBins - 1 ? b : kTopkBins - 1;
 }
 
 template <int CS>
@@ -68,12 +98,13 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(const float *__restrict__
                                                        const int32_t *__restrict__ q_pos, int Tq,
                                                        int nc_max, int k,
                                                        int32_t *__restrict__ idx_out) {
-  extern __shared__ uint32_t keys[];  // [slice]
+  extern __shared__ uint32_t dyn[];
   __shared__ TopkShared sh;
+  constexpr int NT = kTopkThreads;
   const int rank = (CS > 1) ? (int)cg::this_cluster().block_rank() : 0;
   const int r = blockIdx.x / CS;  // clusters tile the grid along x
   const int b = r / Tq, tq = r % Tq;
-  const int tid = threadIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
   int32_t *orow = idx_out + (size_t)r * k;
 
   int t, v = 0;
@@ -84,109 +115,227 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(const float *__restrict__
       v = 0;
     }
   }
-
   // fewer visible entries than k: all of them, then -1 padding
   if (v <= k) {
-    for (int j = rank * kTopkThreads + tid; j < k; j += CS * kTopkThreads) orow[j] = j < v ? j : -1;
+    for (int j = rank * NT + tid; j < k; j += CS * NT) orow[j] = j < v ? j : -1;
     return;  // uniform across the cluster: no barrier was entered
   }
 
-  const int per = (v + CS - 1) / CS;
+  const int per = (v + CS - 1) / CS;  // the same in every CTA of the cluster
   const int lo = min(v, rank * per), hi = min(v, lo + per);
   const int len = hi - lo;
+  uint32_t *keys = dyn;                                         // [per]
+  int *cand_pos = reinterpret_cast<int *>(dyn + per);           // [min(per, cap)]
+  uint32_t *selbits = dyn + per + (per < kTopkRankCap ? per : kTopkRankCap);  // [per/32]
   const float *srow = scores + (size_t)r * nc_max;
-  for (int j = tid; j < len; j += kTopkThreads) keys[j] = order_key(__ldg(srow + lo + j));
 
-  uint32_t pmask = 0u, pval = 0u;  // prefix of T found so far
-  int need = k;                    // keys still needed among those matching the prefix
-  bool all_eq = false;             // every key matching the prefix is selected
-  for (int pass = 0; pass < 4; ++pass) {
-    const int shift = 24 - 8 * pass;
-    int *h = sh.hist[pass & 1];
-    for (int j = tid; j < 256; j += kTopkThreads) h[j] = 0;
+  // ---- A: keys, min / max
+  uint32_t lmin = 0xFFFFFFFFu, lmax = 0u;
+  for (int j = tid; j < len; j += NT) {
+    const uint32_t key = order_key(__ldg(srow + lo + j));
+    keys[j] = key;
+    lmin = min(lmin, key);
+    lmax = max(lmax, key);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    lmin = min(lmin, __shfl_xor_sync(0xffffffffu, lmin, o));
+    lmax = max(lmax, __shfl_xor_sync(0xffffffffu, lmax, o));
+  }
+  if (lane == 0) {
+    sh.red[0][wid] = lmin;
+    sh.red[1][wid] = lmax;
+  }
+  for (int j = tid; j < kTopkBins; j += NT) sh.hist[j] = 0;
+  if (tid == 0) sh.ncand = 0;
+  __syncthreads();
+  if (tid == 0) {
+    uint32_t a = 0xFFFFFFFFu, z = 0u;
+    for (int w = 0; w < NT / 32; ++w) {
+      a = min(a, sh.red[0][w]);
+      z = max(z, sh.red[1][w]);
+    }
+    sh.kmin = a;
+    sh.kmax = z;
+  }
+  cluster_barrier<CS>();
+  uint32_t gmin = 0xFFFFFFFFu, gmax = 0u;
+#pragma unroll
+  for (int c = 0; c < CS; ++c) {
+    const TopkShared *p = peer_ptr<CS>(&sh, c);
+    gmin = min(gmin, p->kmin);
+    gmax = max(gmax, p->kmax);
+  }
+  const float fmin = key_to_float(gmin), fmax = key_to_float(gmax);
+  const float range = __fsub_rn(fmax, fmin);
+  const float scale = (range > 0.f && range <= 3.0e38f) ? __fdiv_rn((float)kTopkBins, range) : 0.f;
+
+  // ---- B: value histogram, the bin b* of the k-th largest key
+  for (int j = tid; j < len; j += NT) atomicAdd(&sh.hist[value_bin(keys[j], fmin, scale)], 1);
+  cluster_barrier<CS>();
+  constexpr int BPT = kTopkBins / NT;  // bins per thread, in descending order
+  int cnt[BPT], mine = 0;
+#pragma unroll
+  for (int i = 0; i < BPT; ++i) {
+    const int bin = kTopkBins - 1 - (BPT * tid + i);
+    int s = 0;
+#pragma unroll
+    for (int c = 0; c < CS; ++c) s += peer_ptr<CS>(&sh, c)->hist[bin];
+    cnt[i] = s;
+    mine += s;
+  }
+  int total;
+  int above = block_exclusive_scan(mine, sh.scan, &total);
+#pragma unroll
+  for (int i = 0; i < BPT; ++i) {
+    if (above < k && above + cnt[i] >= k) {
+      sh.info[0] = kTopkBins - 1 - (BPT * tid + i);
+      sh.info[1] = above;
+      sh.info[2] = cnt[i];
+    }
+    above += cnt[i];
+  }
+  __syncthreads();
+  const int bstar = sh.info[0];
+  const int need = k - sh.info[1];  // keys to take from b*
+  const int incand = sh.info[2];    // keys in b* over the whole row
+  // keys of b*: mode 0 all selected, 1 selected where marked in selbits,
+  // 2 by the radix threshold (pmask, pval), ties by index
+  const int mode = (incand == need) ? 0 : (incand <= kTopkRankCap ? 1 : 2);
+  uint32_t pmask = 0u, pval = 0u;
+  int need_eq = 0;
+  bool all_eq = false;
+
+  if (mode == 1) {
+    // ---- C1: gather every candidate of the cluster, rank this CTA's own
+    for (int j = tid; j < len; j += NT)
+      if (value_bin(keys[j], fmin, scale) == bstar) cand_pos[atomicAdd(&sh.ncand, 1)] = j;
+    for (int j = tid; j < (len + 31) / 32; j += NT) selbits[j] = 0u;
+    cluster_barrier<CS>();
+    int off = 0;
+    for (int c = 0; c < CS; ++c) {
+      const int nc = peer_ptr<CS>(&sh, c)->ncand;
+      const int *pc = peer_ptr<CS>(cand_pos, c);
+      const uint32_t *pk = peer_ptr<CS>(keys, c);
+      const int plo = min(v, c * per);
+      for (int u = tid; u < nc; u += NT) {
+        const int pos = pc[u];
+        sh.all_key[off + u] = pk[pos];
+        sh.all_idx[off + u] = plo + pos;
+      }
+      off += nc;
+    }
     __syncthreads();
-    // warp-aggregated shared-memory histogram: scores crowd into few top
-    // digits, so lanes with the same bin add once through their leader
-    for (int j0 = 0; j0 < len; j0 += kTopkThreads) {
-      const int j = j0 + tid;
-      const uint32_t key = j < len ? keys[j] : 0u;
-      const bool ok = j < len && (key & pmask) == pval;
-      const unsigned act = __ballot_sync(0xffffffffu, ok);
-      if (ok) {
-        const uint32_t bin = (key >> shift) & 255u;
-        const unsigned same = __match_any_sync(act, bin);
-        if ((threadIdx.x & 31) == __ffs(same) - 1) atomicAdd(&h[bin], __popc(same));
+    for (int u = tid; u < sh.ncand; u += NT) {
+      const int pos = cand_pos[u];
+      const uint32_t key = keys[pos];
+      const int gi = lo + pos;
+      int beat = 0;
+      for (int m = 0; m < incand; ++m) {
+        const uint32_t km = sh.all_key[m];
+        beat += (km > key) || (km == key && sh.all_idx[m] < gi);
+      }
+      if (beat < need) atomicOr(&selbits[pos >> 5], 1u << (pos & 31));
+    }
+    __syncthreads();
+  } else if (mode == 2) {
+    // ---- C2: radix select among the keys of b* (degenerate distributions)
+    cluster_barrier<CS>();  // peers are done reading the value histogram
+    need_eq = need;
+    for (int pass = 0; pass < 4; ++pass) {
+      const int shift = 24 - 8 * pass;
+      int *h = sh.hist + 256 * (pass & 1);
+      for (int j = tid; j < 256; j += NT) h[j] = 0;
+      __syncthreads();
+      for (int j0 = 0; j0 < len; j0 += NT) {
+        const int j = j0 + tid;
+        const uint32_t key = j < len ? keys[j] : 0u;
+        const bool ok = j < len && (key & pmask) == pval && value_bin(key, fmin, scale) == bstar;
+        const unsigned act = __ballot_sync(0xffffffffu, ok);
+        if (ok) {
+          const uint32_t bin = (key >> shift) & 255u;
+          const unsigned same = __match_any_sync(act, bin);
+          if (lane == __ffs(same) - 1) atomicAdd(&h[bin], __popc(same));
+        }
+      }
+      cluster_barrier<CS>();
+      int c2 = 0;
+      if (tid < 256) {
+        const int bin = 255 - tid;
+#pragma unroll
+        for (int c = 0; c < CS; ++c) c2 += peer_ptr<CS>(&sh, c)->hist[256 * (pass & 1) + bin];
+      }
+      int tot2;
+      const int ab2 = block_exclusive_scan(c2, sh.scan, &tot2);
+      if (tid < 256 && ab2 < need_eq && ab2 + c2 >= need_eq) {
+        sh.info[0] = 255 - tid;
+        sh.info[1] = ab2;
+        sh.info[2] = c2;
+      }
+      __syncthreads();
+      need_eq -= sh.info[1];
+      pmask |= 255u << shift;
+      pval |= (uint32_t)sh.info[0] << shift;
+      const bool done = (sh.info[2] == need_eq);
+      __syncthreads();  // info is read by every thread before the next pass rewrites it
+      if (done) {
+        all_eq = true;
+        break;
       }
     }
-    cluster_barrier<CS>();
-    // bin totals over the cluster, in fixed rank order; thread j owns bin 255-j
-    int cnt = 0;
-    if (tid < 256) {
-      const int bin = 255 - tid;
-#pragma unroll
-      for (int c = 0; c < CS; ++c) cnt += peer<CS>(&sh, c)->hist[pass & 1][bin];
-    }
-    int total;
-    const int above = block_exclusive_scan(cnt, sh.scan, &total);  // keys in higher bins
-    if (tid < 256 && above < need && above + cnt >= need) {
-      sh.digit_info[0] = 255 - tid;
-      sh.digit_info[1] = above;
-      sh.digit_info[2] = cnt;
-    }
-    __syncthreads();
-    const uint32_t bin = (uint32_t)sh.digit_info[0];
-    need -= sh.digit_info[1];
-    pmask |= 255u << shift;
-    pval |= bin << shift;
-    if (sh.digit_info[2] == need) {
-      all_eq = true;
-      break;
-    }
   }
 
-  // count this CTA's selected keys: greater than the prefix, and equal to it
-  constexpr int NT = kTopkThreads;
+  // ---- D: count, exchange offsets, write in index order
   const int chunk = (len + NT - 1) / NT;
   const int c0 = min(len, tid * chunk), c1 = min(len, c0 + chunk);
-  int n_gt = 0, n_eq = 0;
+  // 1: selected; 2: tied at the radix threshold (mode 2); 0: not selected
+  auto classify = [&](int j) -> int {
+    const uint32_t key = keys[j];
+    const int bn = value_bin(key, fmin, scale);
+    if (bn != bstar) return bn > bstar ? 1 : 0;
+    if (mode == 0) return 1;
+    if (mode == 1) return (int)((selbits[j >> 5] >> (j & 31)) & 1u);
+    const uint32_t km = key & pmask;
+    if (km > pval) return 1;
+    if (km == pval) return all_eq ? 1 : 2;
+    return 0;
+  };
+  int n_sel = 0, n_eq = 0;
   for (int j = c0; j < c1; ++j) {
-    const uint32_t km = keys[j] & pmask;
-    n_gt += km > pval;
-    n_eq += km == pval;
+    const int cl = classify(j);
+    n_sel += cl == 1;
+    n_eq += cl == 2;
   }
-  int cta_gt, cta_eq;
-  const int gt_before = block_exclusive_scan(n_gt, sh.scan, &cta_gt);
+  int cta_sel, cta_eq;
+  block_exclusive_scan(n_sel, sh.scan, &cta_sel);
   const int eq_before = block_exclusive_scan(n_eq, sh.scan, &cta_eq);
   if (tid == 0) {
-    sh.cta_counts[0] = cta_gt;
+    sh.cta_counts[0] = cta_sel;
     sh.cta_counts[1] = cta_eq;
   }
   cluster_barrier<CS>();
-  // output offset of this CTA and the number of its equal keys to take
   int off = 0, eq_seen = 0, take_eq = 0;
 #pragma unroll
   for (int c = 0; c < CS; ++c) {
-    const TopkShared *p = peer<CS>(&sh, c);
+    const TopkShared *p = peer_ptr<CS>(&sh, c);
     const int g = p->cta_counts[0], e = p->cta_counts[1];
-    const int te = all_eq ? e : max(0, min(e, need - eq_seen));
+    const int te = max(0, min(e, need_eq - eq_seen));
     if (c < rank) off += g + te;
     if (c == rank) take_eq = te;
     eq_seen += e;
   }
-  // per-thread: equal keys it takes, then its output position
   const int my_take = max(0, min(n_eq, take_eq - eq_before));
   int dummy;
-  int pos = off + block_exclusive_scan(n_gt + my_take, sh.scan, &dummy);
-  (void)gt_before;
+  int pos = off + block_exclusive_scan(n_sel + my_take, sh.scan, &dummy);
   int eq_rank = eq_before;
   for (int j = c0; j < c1; ++j) {
-    const uint32_t km = keys[j] & pmask;
+    const int cl = classify(j);
     // (pos < k always holds: exactly k keys are selected; the guard keeps a
     // miscount from ever writing outside the row)
-    if (km > pval) {
+    if (cl == 1) {
       if (pos < k) orow[pos] = lo + j;
       ++pos;
-    } else if (km == pval) {
+    } else if (cl == 2) {
       if (eq_rank < take_eq) {
         if (pos < k) orow[pos] = lo + j;
         ++pos;
@@ -194,7 +343,7 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(const float *__restrict__
       ++eq_rank;
     }
   }
-  cluster_barrier<CS>();  // peers may still read this CTA's counts
+  cluster_barrier<CS>();  // peers may still read this CTA's shared memory
 }
 
 }  // namespace csa

@@ -148,7 +148,7 @@ CSA_API int hca_compress(const void *x, const int32_t *lens, int B, int n_max, i
  *   workspace, ws_bytes      >= csa_index_topk_workspace_size(...), 16-byte
  *                            aligned; may be NULL when that size is 0
  * Inputs must be finite.  Supported: (HI, dI) with HI in [1, 128] and dI in
- * {32, 64, 128}; 1 <= k <= 4096; nc_max <= 393216 (1.5M tokens).
+ * {32, 64, 128}; 1 <= k <= 4096; nc_max <= 327680 (1.31M tokens).
  * ---------------------------------------------------------------------- */
 CSA_API size_t csa_index_topk_workspace_size(int B, int Tq, int nc_max, int has_scores_out);
 

@@ -78,7 +78,7 @@ def test_index_topk_validation(L):
     assert idx_call(L, kk=4097) == E_UNSUP
     assert idx_call(L, HI=0) == E_UNSUP
     assert idx_call(L, dI=96) == E_UNSUP
-    assert idx_call(L, nc=393217) == E_UNSUP
+    assert idx_call(L, nc=327681) == E_UNSUP
     assert idx_call(L, w=None) == E_NULL
     assert idx_call(L, q=A4) == E_ALIGN
     assert idx_call(L, ws=None) == E_WS
