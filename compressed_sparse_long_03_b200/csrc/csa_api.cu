@@ -48,12 +48,14 @@ int launch_status(const char *what) {
 }
 
 // Raise a kernel's dynamic shared-memory limit once per (kernel, device).
+// Applied whenever dynamic memory is used: static plus dynamic shared memory
+// above 48 KB needs the opt-in even when the dynamic part alone is smaller.
 std::mutex g_attr_mu;
 std::unordered_map<std::string, size_t> g_attr_done;
 
 template <typename K>
 int ensure_smem(K kernel, size_t bytes, const char *what) {
-  if (bytes <= 48 * 1024) return CSA_OK;
+  if (bytes == 0) return CSA_OK;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return fail(CSA_ERR_CUDA, "%s: cudaGetDevice failed", what);
   char key[64];

@@ -129,14 +129,42 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(const float *__restrict__
   uint32_t *selbits = dyn + per + (per < kTopkRankCap ? per : kTopkRankCap);  // [per/32]
   const float *srow = scores + (size_t)r * nc_max;
 
-  // ---- A: keys, min / max
+  // ---- A: keys, min / max.  Scores stream from L2 as 16-byte vectors, eight
+  // in flight per thread, where the row's alignment allows it.
   uint32_t lmin = 0xFFFFFFFFu, lmax = 0u;
-  for (int j = tid; j < len; j += NT) {
-    const uint32_t key = order_key(__ldg(srow + lo + j));
+  auto take = [&](int j, float f) {
+    const uint32_t key = order_key(f);
     keys[j] = key;
     lmin = min(lmin, key);
     lmax = max(lmax, key);
+  };
+  const float *src = srow + lo;
+  int head = (int)((16 - (reinterpret_cast<uintptr_t>(src) & 15)) & 15) / 4;  // scalars to 16 B
+  head = min(head, len);
+  for (int j = tid; j < head; j += NT) take(j, __ldg(src + j));
+  const int nvec = (len - head) / 4;
+  const float4 *vsrc = reinterpret_cast<const float4 *>(src + head);
+  constexpr int UNR = 8;
+  for (int u0 = 0; u0 < nvec; u0 += NT * UNR) {
+    float4 f[UNR];
+#pragma unroll
+    for (int i = 0; i < UNR; ++i) {
+      const int u = u0 + i * NT + tid;
+      f[i] = u < nvec ? __ldg(vsrc + u) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int i = 0; i < UNR; ++i) {
+      const int u = u0 + i * NT + tid;
+      if (u < nvec) {
+        const int j = head + 4 * u;
+        take(j, f[i].x);
+        take(j + 1, f[i].y);
+        take(j + 2, f[i].z);
+        take(j + 3, f[i].w);
+      }
+    }
   }
+  for (int j = head + 4 * nvec + tid; j < len; j += NT) take(j, __ldg(src + j));
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
     lmin = min(lmin, __shfl_xor_sync(0xffffffffu, lmin, o));
