@@ -48,6 +48,7 @@ __global__ void __launch_bounds__(kAtThreads, 1) k_attend_tc(AttendArgs a) {
   __shared__ uint32_t tmem_holder;
   __shared__ uint64_t bar_s, bar_o;
   __shared__ int kvalid[kAtMaxTile];
+  __shared__ const __nv_bfloat16 *rowp[kAtMaxTile];
   __shared__ float pm[128], pl[128];
   __shared__ float mw[136], minv[128];  // merge weights [head][rank], 1 / sum
   __shared__ int abort_flag;
@@ -129,9 +130,9 @@ __global__ void __launch_bounds__(kAtThreads, 1) k_attend_tc(AttendArgs a) {
   for (int p0 = lo; p0 < hi && alive; p0 += kAtMaxTile) {
     const int ntile = min(kAtMaxTile, hi - p0);
     const int nchunk = (ntile + 31) >> 5;  // 32-key chunks; MMA N = 32 * nchunk
-    // ---- gather the key rows (16 chunks of 16 B each)
-    for (int u = tid; u < nchunk * 32 * 16; u += kAtThreads) {
-      const int j = u >> 4, c = u & 15;
+    // ---- row pointers of the tile's keys (one coalesced index read), then
+    // the rows themselves: 16 chunks of 16 B each, no dependent global loads
+    for (int j = tid; j < nchunk * 32; j += kAtThreads) {
       const int p = p0 + j;
       const __nv_bfloat16 *row = nullptr;
       if (j < ntile) {
@@ -143,7 +144,13 @@ __global__ void __launch_bounds__(kAtThreads, 1) k_attend_tc(AttendArgs a) {
           row = kv_tok + ((size_t)b * a.n_tok + (s % a.n_tok)) * D;
         }
       }
-      if (c == 0) kvalid[j] = row != nullptr;
+      rowp[j] = row;
+      kvalid[j] = row != nullptr;
+    }
+    __syncthreads();
+    for (int u = tid; u < nchunk * 32 * 16; u += kAtThreads) {
+      const int j = u >> 4, c = u & 15;
+      const __nv_bfloat16 *row = rowp[j];
       const uint32_t dst = smem_u32(sK) + (c >> 3) * kAtKHalf + j * 128 + (((c & 7) ^ (j & 7)) << 4);
       cp_async16(dst, row ? row + c * 8 : kv_tok, row ? 16u : 0u);
     }

@@ -56,9 +56,10 @@ struct TopkShared {
 };
 
 // Dynamic shared memory of one CTA for slices of up to `per` keys: the keys,
-// the candidate positions and the selection bit mask.
+// the candidates (key and position) and the selection bit mask.
 __host__ __device__ constexpr size_t topk_dyn_bytes(int per) {
-  return 4ull * ((size_t)per + (size_t)(per < kTopkRankCap ? per : kTopkRankCap) + ((size_t)per + 31) / 32);
+  return 4ull * ((size_t)per + 2 * (size_t)(per < kTopkRankCap ? per : kTopkRankCap) +
+                 ((size_t)per + 31) / 32);
 }
 
 template <int CS>
@@ -124,9 +125,11 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(const float *__restrict__
   const int per = (v + CS - 1) / CS;  // the same in every CTA of the cluster
   const int lo = min(v, rank * per), hi = min(v, lo + per);
   const int len = hi - lo;
+  const int ccap = per < kTopkRankCap ? per : kTopkRankCap;
   uint32_t *keys = dyn;                                         // [per]
-  int *cand_pos = reinterpret_cast<int *>(dyn + per);           // [min(per, cap)]
-  uint32_t *selbits = dyn + per + (per < kTopkRankCap ? per : kTopkRankCap);  // [per/32]
+  uint32_t *cand_key = dyn + per;                               // [ccap]
+  int *cand_pos = reinterpret_cast<int *>(dyn + per + ccap);    // [ccap]
+  uint32_t *selbits = dyn + per + 2 * ccap;                     // [per/32]
   const float *srow = scores + (size_t)r * nc_max;
 
   // ---- A: keys, min / max.  Scores stream from L2 as 16-byte vectors, eight
@@ -236,27 +239,32 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(const float *__restrict__
 
   if (mode == 1) {
     // ---- C1: gather every candidate of the cluster, rank this CTA's own
-    for (int j = tid; j < len; j += NT)
-      if (value_bin(keys[j], fmin, scale) == bstar) cand_pos[atomicAdd(&sh.ncand, 1)] = j;
+    for (int j = tid; j < len; j += NT) {
+      const uint32_t key = keys[j];
+      if (value_bin(key, fmin, scale) == bstar) {
+        const int u = atomicAdd(&sh.ncand, 1);
+        cand_key[u] = key;
+        cand_pos[u] = j;
+      }
+    }
     for (int j = tid; j < (len + 31) / 32; j += NT) selbits[j] = 0u;
     cluster_barrier<CS>();
     int off = 0;
     for (int c = 0; c < CS; ++c) {
       const int nc = peer_ptr<CS>(&sh, c)->ncand;
       const int *pc = peer_ptr<CS>(cand_pos, c);
-      const uint32_t *pk = peer_ptr<CS>(keys, c);
+      const uint32_t *pk = peer_ptr<CS>(cand_key, c);
       const int plo = min(v, c * per);
       for (int u = tid; u < nc; u += NT) {
-        const int pos = pc[u];
-        sh.all_key[off + u] = pk[pos];
-        sh.all_idx[off + u] = plo + pos;
+        sh.all_key[off + u] = pk[u];
+        sh.all_idx[off + u] = plo + pc[u];
       }
       off += nc;
     }
     __syncthreads();
     for (int u = tid; u < sh.ncand; u += NT) {
       const int pos = cand_pos[u];
-      const uint32_t key = keys[pos];
+      const uint32_t key = cand_key[u];
       const int gi = lo + pos;
       int beat = 0;
       for (int m = 0; m < incand; ++m) {
@@ -313,10 +321,11 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(const float *__restrict__
     }
   }
 
-  // ---- D: count, exchange offsets, write in index order
-  const int chunk = (len + NT - 1) / NT;
-  const int c0 = min(len, tid * chunk), c1 = min(len, c0 + chunk);
-  // 1: selected; 2: tied at the radix threshold (mode 2); 0: not selected
+  // ---- D: count, exchange offsets, write in index order.  Warp w owns the
+  // contiguous chunk [w*cw, (w+1)*cw) of the slice and walks it in groups of
+  // 32 consecutive keys (lane = key: conflict-free shared-memory reads);
+  // positions come from ballots within a group and scans across warps.
+  // classify: 1 selected, 2 tied at the radix threshold (mode 2), 0 not
   auto classify = [&](int j) -> int {
     const uint32_t key = keys[j];
     const int bn = value_bin(key, fmin, scale);
@@ -328,15 +337,20 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(const float *__restrict__
     if (km == pval) return all_eq ? 1 : 2;
     return 0;
   };
-  int n_sel = 0, n_eq = 0;
-  for (int j = c0; j < c1; ++j) {
-    const int cl = classify(j);
-    n_sel += cl == 1;
-    n_eq += cl == 2;
+  constexpr int NW = NT / 32;
+  const int cw = ((len + NW - 1) / NW + 31) & ~31;
+  const int w0 = min(len, wid * cw), w1 = min(len, w0 + cw);
+  const unsigned lt = (1u << lane) - 1u;
+  int n_sel = 0, n_eq = 0;  // warp totals (identical in every lane)
+  for (int g = w0; g < w1; g += 32) {
+    const int j = g + lane;
+    const int cl = j < w1 ? classify(j) : 0;
+    n_sel += __popc(__ballot_sync(0xffffffffu, cl == 1));
+    n_eq += __popc(__ballot_sync(0xffffffffu, cl == 2));
   }
   int cta_sel, cta_eq;
-  block_exclusive_scan(n_sel, sh.scan, &cta_sel);
-  const int eq_before = block_exclusive_scan(n_eq, sh.scan, &cta_eq);
+  const int sel_before = block_exclusive_scan(lane == 0 ? n_sel : 0, sh.scan, &cta_sel);
+  const int eq_before = block_exclusive_scan(lane == 0 ? n_eq : 0, sh.scan, &cta_eq);
   if (tid == 0) {
     sh.cta_counts[0] = cta_sel;
     sh.cta_counts[1] = cta_eq;
@@ -352,24 +366,30 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(const float *__restrict__
     if (c == rank) take_eq = te;
     eq_seen += e;
   }
-  const int my_take = max(0, min(n_eq, take_eq - eq_before));
-  int dummy;
-  int pos = off + block_exclusive_scan(n_sel + my_take, sh.scan, &dummy);
-  int eq_rank = eq_before;
-  for (int j = c0; j < c1; ++j) {
-    const int cl = classify(j);
-    // (pos < k always holds: exactly k keys are selected; the guard keeps a
-    // miscount from ever writing outside the row)
-    if (cl == 1) {
-      if (pos < k) orow[pos] = lo + j;
-      ++pos;
-    } else if (cl == 2) {
-      if (eq_rank < take_eq) {
-        if (pos < k) orow[pos] = lo + j;
-        ++pos;
-      }
-      ++eq_rank;
+  // this warp's first output slot: selected keys of earlier warps, plus the
+  // tied keys of earlier warps that are taken
+  const int wsel = __shfl_sync(0xffffffffu, sel_before, 0);
+  const int weq = __shfl_sync(0xffffffffu, eq_before, 0);
+  int pos = off + wsel + max(0, min(weq, take_eq));
+  int eq_rank = weq;
+  for (int g = w0; g < w1; g += 32) {
+    const int j = g + lane;
+    const int cl = j < w1 ? classify(j) : 0;
+    const unsigned ms = __ballot_sync(0xffffffffu, cl == 1);
+    const unsigned me = __ballot_sync(0xffffffffu, cl == 2);
+    // tied keys are taken in index order while eq_rank < take_eq
+    const int te_here = max(0, min(__popc(me), take_eq - eq_rank));
+    unsigned mt = me;  // the first te_here tied keys of this group
+    for (int d = __popc(me) - te_here; d > 0; --d) mt &= ~(1u << (31 - __clz(mt)));
+    const unsigned mall = ms | mt;
+    if ((mall >> lane) & 1u) {
+      const int p = pos + __popc(mall & lt);
+      // (p < k always holds: exactly k keys are selected; the guard keeps a
+      // miscount from ever writing outside the row)
+      if (p < k) orow[p] = lo + j;
     }
+    pos += __popc(mall);
+    eq_rank += __popc(me);
   }
   cluster_barrier<CS>();  // peers may still read this CTA's shared memory
 }
