@@ -83,6 +83,8 @@ __global__ void __launch_bounds__(kAttThreads) k_attend_fma(AttendArgs a) {
   const T *kv_tok = static_cast<const T *>(a.kv_tok);
   T *out = static_cast<T *>(a.out) + (size_t)r * H * D;
 
+  pdl_wait();  // launched with programmatic serialisation: inputs may still be in flight
+  pdl_launch_dependents();
   int t;
   bool ok = query_position(a.lens, a.q_pos, b, a.Tq, tq, t);
   int v = 0, w0 = 0, nwin = 0;

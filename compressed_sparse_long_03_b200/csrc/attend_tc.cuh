@@ -70,6 +70,8 @@ __global__ void __launch_bounds__(kAtThreads, 1) k_attend_tc(AttendArgs a) {
   const __nv_bfloat16 *kv_tok = static_cast<const __nv_bfloat16 *>(a.kv_tok);
   __nv_bfloat16 *out = static_cast<__nv_bfloat16 *>(a.out) + (size_t)r * H * D;
 
+  pdl_wait();
+  pdl_launch_dependents();
   int t;
   bool ok = query_position(a.lens, a.q_pos, b, a.Tq, tq, t);
   int v = 0, w0 = 0, nwin = 0;

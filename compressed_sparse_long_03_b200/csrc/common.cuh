@@ -28,6 +28,18 @@ __device__ int g_dev_err;
 __device__ __forceinline__ void raise_dev_err(int code) { atomicCAS(&g_dev_err, 0, code); }
 
 // ---------------------------------------------------------------------------
+// programmatic dependent launch: a kernel launched with programmatic stream
+// serialisation may start while its predecessor in the stream is finishing.
+// It waits for the predecessor's completion (and memory) before touching
+// global memory, and lets its own dependents launch once all its CTAs run.
+// Both are no-ops for a kernel launched without the attribute.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// ---------------------------------------------------------------------------
 // element conversion
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ float to_f(float v) { return v; }

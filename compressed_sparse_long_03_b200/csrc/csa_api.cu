@@ -73,6 +73,8 @@ int ensure_smem(K kernel, size_t bytes, const char *what) {
 
 // Launch `kernel` on a 1-D grid of clusters of `cs` CTAs (cs == 1: a plain
 // launch).
+// The tensor-core path's kernels are launched with programmatic stream
+// serialisation (they start early and wait in-kernel for their predecessor).
 template <typename... KArgs, typename... Args>
 int launch_cluster(void (*kernel)(KArgs...), int cs, unsigned grid, unsigned block, size_t smem,
                    cudaStream_t stream, const char *what, Args... args) {
@@ -81,15 +83,20 @@ int launch_cluster(void (*kernel)(KArgs...), int cs, unsigned grid, unsigned blo
   cfg.blockDim = dim3(block, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
+  int n = 0;
+  attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[n].val.programmaticStreamSerializationAllowed = 1;
+  ++n;
   if (cs > 1) {
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = cs;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    attr[n].id = cudaLaunchAttributeClusterDimension;
+    attr[n].val.clusterDim.x = cs;
+    attr[n].val.clusterDim.y = 1;
+    attr[n].val.clusterDim.z = 1;
+    ++n;
   }
+  cfg.attrs = attr;
+  cfg.numAttrs = n;
   cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, args...);
   if (e != cudaSuccess) {
     cudaGetLastError();
@@ -257,8 +264,7 @@ int launch_index_tc(const void *qI, const void *w, const void *kI, const int32_t
   a.R = R;
   a.stages = stages;
   a.fill_invisible = fill ? 1 : 0;
-  kern<<<num_sms(), csa::kTcThreads, smem, st>>>(tmK, tmQ, a);
-  return launch_status(what);
+  return launch_cluster(kern, 1, (unsigned)num_sms(), csa::kTcThreads, smem, st, what, tmK, tmQ, a);
 }
 
 template <int DI>

@@ -129,6 +129,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     tmem_alloc(smem_u32(&tmem_holder), TMEM_COLS);
     tmem_relinquish();
   }
+  pdl_wait();  // inputs may come from the previous kernel in the stream
+  pdl_launch_dependents();
 
   // this CTA's contiguous share of the visible tiles
   {

@@ -107,6 +107,8 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(const float *__restrict__
   const int b = r / Tq, tq = r % Tq;
   const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
   int32_t *orow = idx_out + (size_t)r * k;
+  pdl_wait();
+  pdl_launch_dependents();
 
   int t, v = 0;
   if (query_position(lens, q_pos, b, Tq, tq, t)) {
