@@ -166,23 +166,14 @@ def run_ours(args, rank, world, dev):
     s = dict(wl.sizes)
     B, nc, k, window = s["B"], s["nc"], s["k"], s["window"]
     D = {n: to_dev(wl[n], f"cuda:{dev}") for n in ("kI", "kv", "win", "q", "qI", "w", "lens")}
-    scores = torch.empty(B, 1, nc, dtype=torch.float32, device=dev)
     idx = torch.empty(B, 1, k, dtype=torch.int32, device=dev)
     out = torch.empty(B, 1, s["H"], s["d"], dtype=torch.bfloat16, device=dev)
+    ws = csa.index_topk_workspace(B, 1, nc, False, device=dev)  # scores + zeroed histograms
     stream = torch.cuda.current_stream()
 
-    def step(ev=None):
-        if ev is not None:
-            ev[0].record(stream)
-        csa.csa_index_scores(D["qI"], D["w"], D["kI"], D["lens"], scores_out=scores)
-        if ev is not None:
-            ev[1].record(stream)
-        csa.csa_topk(scores, D["lens"], k, idx_out=idx)
-        if ev is not None:
-            ev[2].record(stream)
+    def step():
+        csa.csa_index_topk(D["qI"], D["w"], D["kI"], D["lens"], k, idx_out=idx, workspace=ws)
         csa.csa_attend(D["q"], D["kv"], D["win"], idx, D["lens"], window=window, out=out)
-        if ev is not None:
-            ev[3].record(stream)
 
     launches_per_step = 3
     for _ in range(args.warmup):
@@ -208,17 +199,23 @@ def run_ours(args, rank, world, dev):
     t1.record(stream)
     torch.cuda.synchronize()
     barrier()
-    # per-kernel durations: the same K steps again with an event around each
-    # kernel (these serialise the kernels; used for the per-kernel roofline)
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
+    # per-kernel durations: the same K steps again with the library's kernel
+    # timing on (events around each kernel; this serialises the kernels)
+    stage = {"index_scores": [], "topk": [], "attend": []}
+    csa.set_kernel_timing(True)
     for i in range(K):
-        step(evs[i])
+        csa.csa_index_topk(D["qI"], D["w"], D["kI"], D["lens"], k, idx_out=idx, workspace=ws)
+        t_idx = csa.kernel_timing()
+        csa.csa_attend(D["q"], D["kv"], D["win"], idx, D["lens"], window=window, out=out)
+        t_att = csa.kernel_timing()
+        stage["index_scores"].append(t_idx[0])
+        stage["topk"].append(t_idx[1])
+        stage["attend"].append(t_att[0])
+    csa.set_kernel_timing(False)
     torch.cuda.synchronize()
     clocks = sampler.stop() if rank == 0 else None
     csa.check_device_error()
     ms = t0.elapsed_time(t1) / K
-    stage = {name: [evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(K)]
-             for j, name in enumerate(("index_scores", "topk", "attend"))}
 
     # end to end through the public API from pinned host buffers: H2D of the
     # step's query inputs, the three calls, D2H of the output
@@ -358,8 +355,8 @@ def main():
                      "peak": hbm_peak, "unit": "GB/s", "frac": achieved / hbm_peak,
                      "traffic": None, "bytes_per_launch": kb, "peak_source": peaks["source"]},
         "stages_us": {k: statistics.median(1000 * x for x in v) for k, v in r["stage"].items()},
-        "stages_note": "per-kernel medians from a second pass of the K steps with an event "
-                       "around each kernel (serialised); ms_per_step is the event-free pass",
+        "stages_note": "per-kernel medians from a second pass of the K steps with the "
+                       "library's kernel timing on (serialised); ms_per_step is the event-free pass",
         "e2e": {"value": e2e, "unit": UNIT, "h2d_bytes_per_step": r["h2d"],
                 "d2h_bytes_per_step": r["d2h"]},
         "gpu_launches": r["launches"],

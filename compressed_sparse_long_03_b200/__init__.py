@@ -47,6 +47,10 @@ def lib() -> ctypes.CDLL:
         L = ctypes.CDLL(LIB_PATH)
         P, I, F, S = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
         L.csa_version.restype = I
+        L.csa_set_kernel_timing.argtypes = [I]
+        L.csa_set_kernel_timing.restype = I
+        L.csa_kernel_timing.argtypes = [ctypes.POINTER(ctypes.c_float), I]
+        L.csa_kernel_timing.restype = I
         L.csa_last_error.restype = ctypes.c_char_p
         L.csa_check_device_error.argtypes = [P]
         L.csa_compress.argtypes = [P, P, I, I, I, P, P, P, I, P, P]
@@ -136,6 +140,29 @@ def index_topk_workspace_size(B, Tq, nc_max, has_scores_out=False) -> int:
     return int(lib().csa_index_topk_workspace_size(B, Tq, nc_max, int(bool(has_scores_out))))
 
 
+def index_topk_workspace(B, Tq, nc_max, has_scores_out=False, device="cuda"):
+    """A zero-filled workspace for csa_index_topk (reusable across calls on
+    one stream: each call leaves its histogram part zero again)."""
+    n = index_topk_workspace_size(B, Tq, nc_max, has_scores_out)
+    return torch.zeros(max(n, 16), dtype=torch.uint8, device=device)
+
+
+def set_kernel_timing(enable: bool) -> None:
+    """Record CUDA events around every kernel of subsequent calls on this
+    host thread (serialises them; for per-kernel measurements)."""
+    _check(lib().csa_set_kernel_timing(int(bool(enable))))
+
+
+def kernel_timing(max_kernels: int = 16):
+    """Durations (ms) of the kernels launched by the last call on this host
+    thread, in launch order (needs set_kernel_timing(True))."""
+    buf = (ctypes.c_float * max_kernels)()
+    n = lib().csa_kernel_timing(buf, max_kernels)
+    if n < 0:
+        raise CsaError(n, last_error())
+    return [buf[i] for i in range(min(n, max_kernels))]
+
+
 def csa_index_topk(q_idx, w, k_idx, lens, k, q_pos=None, idx_out=None, scores_out=None,
                    workspace=None, stream=None):
     """q_idx [B][Tq][HI][dI], w [B][Tq][HI], k_idx [B][nc_max][dI]
@@ -147,7 +174,7 @@ def csa_index_topk(q_idx, w, k_idx, lens, k, q_pos=None, idx_out=None, scores_ou
         idx_out = torch.empty(B, Tq, k, dtype=torch.int32, device=q_idx.device)
     need = index_topk_workspace_size(B, Tq, nc_max, scores_out is not None)
     if workspace is None and need:
-        workspace = torch.empty(need, dtype=torch.uint8, device=q_idx.device)
+        workspace = index_topk_workspace(B, Tq, nc_max, scores_out is not None, q_idx.device)
     ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
     _check(lib().csa_index_topk(_p(q_idx), _p(w), _p(k_idx), _i32(lens), _i32(q_pos), B, Tq, HI, dI,
                                 nc_max, k, _dt(q_idx), _i32(idx_out), _p(scores_out), _p(workspace),

@@ -94,6 +94,12 @@ __device__ __forceinline__ uint32_t order_key(float f) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
+// Histogram bin of a score for the top-k threshold search: the 12 leading
+// bits of its order key (sign, exponent, 3 mantissa bits), so bins are
+// monotone in the score and about 1/8 octave wide.
+constexpr int kScoreBins = 4096;
+__device__ __forceinline__ int score_bin(uint32_t key) { return (int)(key >> 20); }
+
 __device__ __forceinline__ float warp_max(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));

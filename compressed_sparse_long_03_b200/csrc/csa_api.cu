@@ -14,6 +14,7 @@
 #include <mutex>
 #include <string>
 #include <unordered_map>
+#include <vector>
 
 #include "csa.h"
 
@@ -40,6 +41,44 @@ int fail(int code, const char *fmt, ...) {
 }
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// ---------------------------------------------------------------------------
+// optional per-kernel timing (csa_set_kernel_timing): CUDA events recorded
+// on the call's stream around every kernel the call launches
+// ---------------------------------------------------------------------------
+struct TimingSlot {
+  cudaEvent_t a = nullptr, b = nullptr;
+  int dev = -1;
+};
+thread_local bool g_timing = false;
+thread_local std::vector<TimingSlot> g_slots;
+thread_local int g_nlaunch = 0;
+
+void begin_call() { g_nlaunch = 0; }
+
+struct KernelTimer {
+  cudaStream_t st;
+  int slot = -1;
+  explicit KernelTimer(cudaStream_t s) : st(s) {
+    if (!g_timing) return;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if ((int)g_slots.size() <= g_nlaunch) g_slots.resize(g_nlaunch + 1);
+    TimingSlot &ts = g_slots[g_nlaunch];
+    if (ts.dev != dev) {
+      if (ts.a) cudaEventDestroy(ts.a);
+      if (ts.b) cudaEventDestroy(ts.b);
+      cudaEventCreate(&ts.a);
+      cudaEventCreate(&ts.b);
+      ts.dev = dev;
+    }
+    slot = g_nlaunch++;
+    cudaEventRecord(ts.a, st);
+  }
+  ~KernelTimer() {
+    if (slot >= 0) cudaEventRecord(g_slots[slot].b, st);
+  }
+};
 
 int launch_status(const char *what) {
   cudaError_t e = cudaGetLastError();
@@ -97,6 +136,7 @@ int launch_cluster(void (*kernel)(KArgs...), int cs, unsigned grid, unsigned blo
   }
   cfg.attrs = attr;
   cfg.numAttrs = n;
+  KernelTimer timer(stream);
   cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, args...);
   if (e != cudaSuccess) {
     cudaGetLastError();
@@ -190,6 +230,7 @@ int launch_csa_compress(const void *x, const int32_t *lens, int B, int n_max, in
   auto Bw = static_cast<const T *>(Wb);
   auto Z = static_cast<const T *>(b8);
   auto O = static_cast<T *>(out);
+  KernelTimer timer(st);
   switch (d) {
     case 32: csa::k_csa_compress<T, 32><<<grid, 32, 0, st>>>(X, lens, n_max, A, Bw, Z, O, nc_max); break;
     case 64: csa::k_csa_compress<T, 64><<<grid, 64, 0, st>>>(X, lens, n_max, A, Bw, Z, O, nc_max); break;
@@ -207,6 +248,7 @@ int launch_hca_compress(const void *x, const int32_t *lens, int B, int n_max, in
   auto Wp = static_cast<const T *>(W);
   auto Z = static_cast<const T *>(bias);
   auto O = static_cast<T *>(out);
+  KernelTimer timer(st);
   switch (d) {
     case 32: csa::k_hca_compress<T, 32><<<grid, 32, 0, st>>>(X, lens, n_max, m, Wp, Z, O, nc_max); break;
     case 64: csa::k_hca_compress<T, 64><<<grid, 64, 0, st>>>(X, lens, n_max, m, Wp, Z, O, nc_max); break;
@@ -229,6 +271,7 @@ int launch_index_fma(const void *qI, const void *w, const void *kI, const int32_
   int rc = ensure_smem(kern, smem, "csa_index_topk");
   if (rc) return rc;
   dim3 grid(tiles, R);
+  KernelTimer timer(st);
   kern<<<grid, csa::kIdxFmaTile, smem, st>>>(static_cast<const T *>(qI), static_cast<const T *>(w),
                                              static_cast<const T *>(kI), lens, q_pos, Tq, HI,
                                              nc_max, scores);
@@ -238,7 +281,7 @@ int launch_index_fma(const void *qI, const void *w, const void *kI, const int32_
 template <int N, int DI>
 int launch_index_tc(const void *qI, const void *w, const void *kI, const int32_t *lens,
                     const int32_t *q_pos, int R, int Tq, int HI, int nc_max, float *scores,
-                    bool fill, cudaStream_t st) {
+                    bool fill, int *hist, cudaStream_t st) {
   const char *what = "csa_index_scores";
   CUtensorMap tmK, tmQ;
   const int B = R / Tq;
@@ -248,7 +291,7 @@ int launch_index_tc(const void *qI, const void *w, const void *kI, const int32_t
   if (rc) return rc;
   constexpr size_t A_STAGE = (size_t)csa::kTcRows * DI * 2, B_SLOT = (size_t)N * DI * 2;
   const size_t budget = 227 * 1024 - 1024 - 2 * B_SLOT - 1024;  // align slack, barriers, statics
-  const int stages = (int)std::min<size_t>(6, budget / A_STAGE);
+  const int stages = (int)std::min<size_t>(5, budget / A_STAGE);
   const size_t smem = 1024 + stages * A_STAGE + 2 * B_SLOT + 8 * (2 * stages + 9);
   auto kern = csa::k_index_score_tc<N, DI>;
   rc = ensure_smem(kern, smem, what);
@@ -264,29 +307,30 @@ int launch_index_tc(const void *qI, const void *w, const void *kI, const int32_t
   a.R = R;
   a.stages = stages;
   a.fill_invisible = fill ? 1 : 0;
+  a.hist = hist;
   return launch_cluster(kern, 1, (unsigned)num_sms(), csa::kTcThreads, smem, st, what, tmK, tmQ, a);
 }
 
 template <int DI>
 int launch_index_tc_n(const void *qI, const void *w, const void *kI, const int32_t *lens,
                       const int32_t *q_pos, int R, int Tq, int HI, int nc_max, float *scores,
-                      bool fill, cudaStream_t st) {
-  if (HI <= 16) return launch_index_tc<16, DI>(qI, w, kI, lens, q_pos, R, Tq, HI, nc_max, scores, fill, st);
-  if (HI <= 32) return launch_index_tc<32, DI>(qI, w, kI, lens, q_pos, R, Tq, HI, nc_max, scores, fill, st);
-  if (HI <= 64) return launch_index_tc<64, DI>(qI, w, kI, lens, q_pos, R, Tq, HI, nc_max, scores, fill, st);
-  return launch_index_tc<128, DI>(qI, w, kI, lens, q_pos, R, Tq, HI, nc_max, scores, fill, st);
+                      bool fill, int *hist, cudaStream_t st) {
+  if (HI <= 16) return launch_index_tc<16, DI>(qI, w, kI, lens, q_pos, R, Tq, HI, nc_max, scores, fill, hist, st);
+  if (HI <= 32) return launch_index_tc<32, DI>(qI, w, kI, lens, q_pos, R, Tq, HI, nc_max, scores, fill, hist, st);
+  if (HI <= 64) return launch_index_tc<64, DI>(qI, w, kI, lens, q_pos, R, Tq, HI, nc_max, scores, fill, hist, st);
+  return launch_index_tc<128, DI>(qI, w, kI, lens, q_pos, R, Tq, HI, nc_max, scores, fill, hist, st);
 }
 
 template <int CS>
-int launch_topk(const float *scores, const int32_t *lens, const int32_t *q_pos, int R, int Tq,
-                int nc_max, int k, int32_t *idx_out, cudaStream_t st) {
+int launch_topk(const float *scores, int *hist, const int32_t *lens, const int32_t *q_pos, int R,
+                int Tq, int nc_max, int k, int32_t *idx_out, cudaStream_t st) {
   const int per = (nc_max + CS - 1) / CS;
   const size_t smem = csa::topk_dyn_bytes(per > 0 ? per : 1);
   auto kern = csa::k_topk<CS>;
   int rc = ensure_smem(kern, smem, "csa_index_topk");
   if (rc) return rc;
   return launch_cluster(kern, CS, (unsigned)CS * R, csa::kTopkThreads, smem, st,
-                        "csa_index_topk (select)", scores, lens, q_pos, Tq, nc_max, k, idx_out);
+                        "csa_index_topk (select)", scores, hist, lens, q_pos, Tq, nc_max, k, idx_out);
 }
 
 // ---------------------------------------------------------------------------
@@ -381,7 +425,22 @@ int attend_common(const void *q, const void *kv_c, const void *kv_tok, int n_tok
 // ===========================================================================
 extern "C" {
 
-int csa_version(void) { return (0 << 16) | 1; }
+int csa_version(void) { return (0 << 16) | 2; }
+
+int csa_set_kernel_timing(int enable) {
+  g_timing = enable != 0;
+  return CSA_OK;
+}
+
+int csa_kernel_timing(float *ms, int max_kernels) {
+  const int n = g_nlaunch;
+  for (int i = 0; i < n && i < max_kernels && ms; ++i) {
+    cudaError_t e = cudaEventSynchronize(g_slots[i].b);
+    if (e == cudaSuccess) e = cudaEventElapsedTime(&ms[i], g_slots[i].a, g_slots[i].b);
+    if (e != cudaSuccess) return fail(CSA_ERR_CUDA, "kernel timing: %s", cudaGetErrorString(e));
+  }
+  return n;
+}
 
 const char *csa_last_error(void) { return g_last_error.c_str(); }
 
@@ -403,6 +462,7 @@ int csa_check_device_error(void *stream) {
 
 int csa_compress(const void *x, const int32_t *lens, int B, int n_max, int d, const void *W_a,
                  const void *W_b, const void *bias8, csa_dtype dt, void *out, void *stream) {
+  begin_call();
   const char *what = "csa_compress";
   int rc = check_dtype(dt, what);
   if (rc) return rc;
@@ -420,6 +480,7 @@ int csa_compress(const void *x, const int32_t *lens, int B, int n_max, int d, co
 
 int hca_compress(const void *x, const int32_t *lens, int B, int n_max, int d, int m, const void *W,
                  const void *bias, csa_dtype dt, void *out, void *stream) {
+  begin_call();
   const char *what = "hca_compress";
   int rc = check_dtype(dt, what);
   if (rc) return rc;
@@ -437,27 +498,32 @@ int hca_compress(const void *x, const int32_t *lens, int B, int n_max, int d, in
 }
 
 size_t csa_index_topk_workspace_size(int B, int Tq, int nc_max, int has_scores_out) {
-  if (B <= 0 || Tq <= 0 || nc_max <= 0 || has_scores_out) return 0;
-  const size_t bytes = sizeof(float) * (size_t)B * Tq * nc_max;
-  return (bytes + 255) & ~(size_t)255;
+  if (B <= 0 || Tq <= 0 || nc_max <= 0) return 0;
+  const long R = (long)B * Tq;
+  size_t bytes = (((size_t)(has_scores_out ? 0 : sizeof(float) * (size_t)R * nc_max)) + 255) & ~(size_t)255;
+  if (R <= 1024) bytes += sizeof(int) * (size_t)R * csa::kScoreBins;  // zero-filled histograms
+  return bytes;
 }
 
 }  // extern "C"
 
 namespace {
 
+// The tensor-core scoring kernel serves bf16 keys of 64 or 128 dims.
+bool index_uses_tc(csa_dtype dt, int dI) { return dt == CSA_BF16 && (dI == 64 || dI == 128); }
+
 int index_scores_impl(const void *q_idx, const void *w, const void *k_idx, const int32_t *lens,
                       const int32_t *q_pos, int B, int Tq, int HI, int dI, int nc_max,
-                      csa_dtype dt, float *scores, bool fill, cudaStream_t st) {
+                      csa_dtype dt, float *scores, bool fill, int *hist, cudaStream_t st) {
   const int R = B * Tq;
   if (R == 0 || nc_max == 0) return CSA_OK;
   if (R > 65535) return fail(CSA_ERR_UNSUPPORTED, "csa_index_scores: B*Tq=%d > 65535", R);
   // bf16 with 128-byte key rows or wider: the tensor-core kernel
-  if (dt == CSA_BF16 && (dI == 64 || dI == 128)) {
+  if (index_uses_tc(dt, dI)) {
     if ((long)B * nc_max >= (1L << 31) || (long)R * HI >= (1L << 31))
       return fail(CSA_ERR_UNSUPPORTED, "csa_index_scores: tensor too large for 32-bit coordinates");
-    return dI == 64 ? launch_index_tc_n<64>(q_idx, w, k_idx, lens, q_pos, R, Tq, HI, nc_max, scores, fill, st)
-                    : launch_index_tc_n<128>(q_idx, w, k_idx, lens, q_pos, R, Tq, HI, nc_max, scores, fill, st);
+    return dI == 64 ? launch_index_tc_n<64>(q_idx, w, k_idx, lens, q_pos, R, Tq, HI, nc_max, scores, fill, hist, st)
+                    : launch_index_tc_n<128>(q_idx, w, k_idx, lens, q_pos, R, Tq, HI, nc_max, scores, fill, hist, st);
   }
   if (dt == CSA_F32) {
     switch (dI) {
@@ -473,16 +539,24 @@ int index_scores_impl(const void *q_idx, const void *w, const void *k_idx, const
   }
 }
 
-int topk_impl(const float *scores, const int32_t *lens, const int32_t *q_pos, int B, int Tq,
-              int nc_max, int k, int32_t *idx_out, cudaStream_t st) {
+int topk_impl(const float *scores, int *hist, const int32_t *lens, const int32_t *q_pos, int B,
+              int Tq, int nc_max, int k, int32_t *idx_out, cudaStream_t st) {
   const int R = B * Tq;
   if (R == 0) return CSA_OK;
   switch (topk_cluster_size(nc_max)) {
-    case 1: return launch_topk<1>(scores, lens, q_pos, R, Tq, nc_max, k, idx_out, st);
-    case 2: return launch_topk<2>(scores, lens, q_pos, R, Tq, nc_max, k, idx_out, st);
-    case 4: return launch_topk<4>(scores, lens, q_pos, R, Tq, nc_max, k, idx_out, st);
-    default: return launch_topk<8>(scores, lens, q_pos, R, Tq, nc_max, k, idx_out, st);
+    case 1: return launch_topk<1>(scores, hist, lens, q_pos, R, Tq, nc_max, k, idx_out, st);
+    case 2: return launch_topk<2>(scores, hist, lens, q_pos, R, Tq, nc_max, k, idx_out, st);
+    case 4: return launch_topk<4>(scores, hist, lens, q_pos, R, Tq, nc_max, k, idx_out, st);
+    default: return launch_topk<8>(scores, hist, lens, q_pos, R, Tq, nc_max, k, idx_out, st);
   }
+}
+
+// Rows up to this count get the score histogram built by the scoring kernel.
+constexpr long kHistMaxRows = 1024;
+
+size_t scores_ws_bytes(int B, int Tq, int nc_max, int has_scores_out) {
+  if (has_scores_out) return 0;
+  return ((sizeof(float) * (size_t)B * Tq * nc_max) + 255) & ~(size_t)255;
 }
 
 // shared argument checks of the indexer entry points
@@ -515,6 +589,7 @@ int csa_index_scores(const void *q_idx, const void *w, const void *k_idx, const 
                      const int32_t *q_pos, int B, int Tq, int HI, int dI, int nc_max,
                      csa_dtype dt, float *scores_out, void *stream) {
   const char *what = "csa_index_scores";
+  begin_call();
   int rc = check_index_args(what, dt, B, Tq, HI, dI, nc_max);
   if (rc) return rc;
   if ((long)B * Tq == 0 || nc_max == 0) return CSA_OK;
@@ -523,18 +598,20 @@ int csa_index_scores(const void *q_idx, const void *w, const void *k_idx, const 
   if (!aligned16(q_idx) || !aligned16(w) || !aligned16(k_idx) || !aligned16(scores_out))
     return fail(CSA_ERR_ALIGN, "%s: tensors must be 16-byte aligned", what);
   return index_scores_impl(q_idx, w, k_idx, lens, q_pos, B, Tq, HI, dI, nc_max, dt, scores_out,
-                           true, static_cast<cudaStream_t>(stream));
+                           true, nullptr, static_cast<cudaStream_t>(stream));
 }
 
 int csa_topk(const float *scores, const int32_t *lens, const int32_t *q_pos, int B, int Tq,
              int nc_max, int k, int32_t *idx_out, void *stream) {
   const char *what = "csa_topk";
+  begin_call();
   int rc = check_topk_args(what, B, Tq, nc_max, k);
   if (rc) return rc;
   if ((long)B * Tq == 0) return CSA_OK;
   if (!lens || !idx_out || (nc_max > 0 && !scores)) return fail(CSA_ERR_NULL, "%s: a required pointer is NULL", what);
   if (scores && !aligned16(scores)) return fail(CSA_ERR_ALIGN, "%s: scores must be 16-byte aligned", what);
-  return topk_impl(scores, lens, q_pos, B, Tq, nc_max, k, idx_out, static_cast<cudaStream_t>(stream));
+  return topk_impl(scores, nullptr, lens, q_pos, B, Tq, nc_max, k, idx_out,
+                   static_cast<cudaStream_t>(stream));
 }
 
 int csa_index_topk(const void *q_idx, const void *w, const void *k_idx, const int32_t *lens,
@@ -542,6 +619,7 @@ int csa_index_topk(const void *q_idx, const void *w, const void *k_idx, const in
                    csa_dtype dt, int32_t *idx_out, float *scores_out, void *workspace,
                    size_t ws_bytes, void *stream) {
   const char *what = "csa_index_topk";
+  begin_call();
   int rc = check_index_args(what, dt, B, Tq, HI, dI, nc_max);
   if (rc) return rc;
   rc = check_topk_args(what, B, Tq, nc_max, k);
@@ -559,15 +637,23 @@ int csa_index_topk(const void *q_idx, const void *w, const void *k_idx, const in
   if (need > 0 && !aligned16(workspace)) return fail(CSA_ERR_ALIGN, "%s: workspace must be 16-byte aligned", what);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   float *scores = scores_out ? scores_out : static_cast<float *>(workspace);
+  // the scoring kernel histograms the scores for the top-k when the rows are
+  // few enough; the histogram part of the workspace is zero on entry and
+  // the top-k kernel clears it again
+  int *hist = nullptr;
+  if (nc_max > 0 && (long)B * Tq <= kHistMaxRows && index_uses_tc(dt, dI))
+    hist = reinterpret_cast<int *>(static_cast<char *>(workspace) +
+                                   scores_ws_bytes(B, Tq, nc_max, scores_out != nullptr));
   rc = index_scores_impl(q_idx, w, k_idx, lens, q_pos, B, Tq, HI, dI, nc_max, dt, scores,
-                         scores_out != nullptr, st);
+                         scores_out != nullptr, hist, st);
   if (rc) return rc;
-  return topk_impl(scores, lens, q_pos, B, Tq, nc_max, k, idx_out, st);
+  return topk_impl(scores, hist, lens, q_pos, B, Tq, nc_max, k, idx_out, st);
 }
 
 int csa_attend(const void *q, const void *kv_c, const void *kv_tok, int n_tok, const int32_t *idx,
                const int32_t *lens, const int32_t *q_pos, int B, int Tq, int H, int d, int nc_max,
                int k, int window, float scale, csa_dtype dt, void *out, void *stream) {
+  begin_call();
   if (k < 1 || k > 4096) return fail(CSA_ERR_UNSUPPORTED, "csa_attend: k=%d not in [1,4096]", k);
   if (!idx && (long)B * Tq > 0) return fail(CSA_ERR_NULL, "csa_attend: idx is NULL");
   return attend_common(q, kv_c, kv_tok, n_tok, idx, lens, q_pos, B, Tq, H, d, nc_max, k, 4, window,
@@ -577,6 +663,7 @@ int csa_attend(const void *q, const void *kv_c, const void *kv_tok, int n_tok, c
 int hca_attend(const void *q, const void *kv_c, const void *kv_tok, int n_tok,
                const int32_t *lens, const int32_t *q_pos, int B, int Tq, int H, int d, int nc_max,
                int m, int window, float scale, csa_dtype dt, void *out, void *stream) {
+  begin_call();
   if (m < 1 || m > 4096) return fail(CSA_ERR_UNSUPPORTED, "hca_attend: m=%d not in [1,4096]", m);
   if (nc_max > 65536) return fail(CSA_ERR_UNSUPPORTED, "hca_attend: nc_max=%d > 65536", nc_max);
   return attend_common(q, kv_c, kv_tok, n_tok, nullptr, lens, q_pos, B, Tq, H, d, nc_max, 0, m,

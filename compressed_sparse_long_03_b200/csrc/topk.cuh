@@ -7,24 +7,29 @@
 // the order (score desc, index asc): ties go to the lower index; -0.0 ranks
 // as +0.0; every visible entry when fewer than k.
 //
-// Design (cluster of CS CTAs per row; no global scratch; no spin waits):
+// Design (cluster of CS CTAs per row; no spin waits):
 //  A. each CTA loads a contiguous slice of the row's visible scores into
-//     shared memory as order-preserving u32 keys and reduces their min/max;
-//     the cluster agrees on the row's [min, max];
-//  B. a 2048-bin histogram whose bins split [min, max] evenly by value.  The
-//     bin function is monotone in the score (round-to-nearest subtract and
-//     multiply are monotone), so bins order keys exactly: the bin b* holding
-//     the k-th largest key, and the count above it, decide every key outside
-//     b*.  Bins by value (not by leading bits) keep the shared-memory atomics
-//     free of hot spots, because fp32 scores share their leading bits;
-//  C. the few keys inside b* ("candidates") are ranked exactly: every CTA
-//     reads all candidates of the cluster through distributed shared memory
-//     and counts, for each of its own, the candidates that beat it under
-//     (score desc, index asc).  When b* holds too many keys for that (a
-//     degenerate distribution, e.g. all scores equal), an MSB-first 8-bit
-//     radix select over the keys of b* takes over;
-//  D. per-CTA counts of selected keys give each CTA its output offset, and
-//     each CTA writes its selected indices in order.
+//     shared memory as order-preserving u32 keys;
+//  B. a histogram over monotone bins of the keys finds the bin b* holding the
+//     k-th largest key and the count above it, which decides every key
+//     outside b*.  Two binnings:
+//       - precomputed (csa_index_topk): the scoring kernel already added each
+//         visible score to a per-row histogram of the 12 leading order-key
+//         bits; every CTA reads that row, then the cluster clears it again;
+//       - in-kernel (csa_topk on caller scores): the cluster agrees on the
+//         row's [min, max] and histograms 2048 bins that split it evenly by
+//         value (round-to-nearest subtract and multiply are monotone).
+//     Both avoid the hot spots of a leading-8-bit radix digit, which fp32
+//     scores mostly share;
+//  C. the keys inside b* ("candidates") are ranked exactly: every CTA reads
+//     all candidates of the cluster through distributed shared memory and
+//     counts, for each of its own, the candidates that beat it under (score
+//     desc, index asc).  When b* holds too many keys for that (a degenerate
+//     distribution, e.g. all scores equal) an MSB-first radix select over the
+//     remaining key bits takes over, ties resolved by index;
+//  D. warp-contiguous 32-key groups: ballots give each selected key its slot,
+//     per-warp and per-CTA counts (exchanged in the cluster) give the
+//     offsets, and the indices come out in ascending order.
 // All decisions are integer comparisons on the same keys in every CTA, so
 // the result is bit-exact and independent of the launch configuration.
 #pragma once
@@ -38,19 +43,19 @@ namespace csa {
 namespace cg = cooperative_groups;
 
 constexpr int kTopkThreads = 512;
-constexpr int kTopkSliceCap = 40960;  // keys per CTA held in shared memory
+constexpr int kTopkSliceCap = 40960;   // keys per CTA held in shared memory
 constexpr int kTopkMaxCluster = 8;
-constexpr int kTopkBins = 2048;
-constexpr int kTopkRankCap = 512;     // candidates of a row ranked directly
+constexpr int kTopkValueBins = 2048;   // in-kernel value histogram
+constexpr int kTopkRankCap = 2048;     // candidates of a row ranked directly
 
 struct TopkShared {
-  int hist[kTopkBins];
+  int hist[kTopkValueBins];  // value histogram, later the radix digit histograms
   int scan[33];
-  uint32_t red[2][kTopkThreads / 32];  // per-warp min / max
-  uint32_t kmin, kmax;                 // this CTA's min / max key
-  int info[4];                         // [0] bin, [1] count above it, [2] count in it
-  int ncand;                           // this CTA's candidates (keys in b*)
-  int cta_counts[2];                   // this CTA's (selected, tied) counts
+  uint32_t red[2][kTopkThreads / 32];
+  uint32_t kmin, kmax;       // this CTA's min / max key
+  int info[4];               // [0] bin, [1] count above it, [2] count in it
+  int ncand;                 // this CTA's candidates (keys in b*)
+  int cta_counts[2];         // this CTA's (selected, tied) counts
   uint32_t all_key[kTopkRankCap];
   int all_idx[kTopkRankCap];
 };
@@ -85,16 +90,50 @@ __device__ __forceinline__ float key_to_float(uint32_t k) {
   return __uint_as_float(u);
 }
 
-// Monotone value bin of a key in [fmin, fmax] (scale = bins / (fmax - fmin);
-// scale == 0 puts every key in bin 0).
-__device__ __forceinline__ int value_bin(uint32_t key, float fmin, float scale) {
-  const float x = __fmul_rn(__fsub_rn(key_to_float(key), fmin), scale);
-  const int b = (int)x;  // x >= 0
-  return b < kTopkBins - 1 ? b : kTopkBins - 1;
+// Monotone bins of the order keys.
+struct Binner {
+  bool fixed;   // score_bin (12 leading key bits) or value bins over [fmin, fmax]
+  float fmin;   // value bins: lower edge
+  float scale;  // value bins: bins / (fmax - fmin); 0 puts every key in bin 0
+  __device__ __forceinline__ int operator()(uint32_t key) const {
+    if (fixed) return score_bin(key);
+    const float x = __fmul_rn(__fsub_rn(key_to_float(key), fmin), scale);
+    const int b = (int)x;  // x >= 0
+    return b < kTopkValueBins - 1 ? b : kTopkValueBins - 1;
+  }
+};
+
+// Bin b* of the k-th largest key given per-bin counts (descending search;
+// BPT bins per thread).  Writes sh.info = {b*, count above, count in b*}.
+template <int NB, typename CountFn>
+__device__ __forceinline__ void find_threshold_bin(TopkShared &sh, int k, CountFn count_of) {
+  constexpr int BPT = NB / kTopkThreads;
+  const int tid = threadIdx.x;
+  int cnt[BPT], mine = 0;
+#pragma unroll
+  for (int i = 0; i < BPT; ++i) {
+    cnt[i] = count_of(NB - 1 - (BPT * tid + i));
+    mine += cnt[i];
+  }
+  int total;
+  int above = block_exclusive_scan(mine, sh.scan, &total);
+#pragma unroll
+  for (int i = 0; i < BPT; ++i) {
+    if (above < k && above + cnt[i] >= k) {
+      sh.info[0] = NB - 1 - (BPT * tid + i);
+      sh.info[1] = above;
+      sh.info[2] = cnt[i];
+    }
+    above += cnt[i];
+  }
+  __syncthreads();
 }
 
+// idx_out row r: the k selected visible entries, ascending.  hist != nullptr:
+// per-row score_bin histograms of the visible scores (cleared on the way).
 template <int CS>
 __global__ void __launch_bounds__(kTopkThreads) k_topk(const float *__restrict__ scores,
+                                                       int *__restrict__ hist,
                                                        const int32_t *__restrict__ lens,
                                                        const int32_t *__restrict__ q_pos, int Tq,
                                                        int nc_max, int k,
@@ -107,6 +146,7 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(const float *__restrict__
   const int b = r / Tq, tq = r % Tq;
   const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
   int32_t *orow = idx_out + (size_t)r * k;
+  int *hrow = hist ? hist + (size_t)r * kScoreBins : nullptr;
   pdl_wait();
   pdl_launch_dependents();
 
@@ -121,6 +161,8 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(const float *__restrict__
   // fewer visible entries than k: all of them, then -1 padding
   if (v <= k) {
     for (int j = rank * NT + tid; j < k; j += CS * NT) orow[j] = j < v ? j : -1;
+    if (hrow)
+      for (int j = rank * NT + tid; j < kScoreBins; j += CS * NT) hrow[j] = 0;
     return;  // uniform across the cluster: no barrier was entered
   }
 
@@ -134,8 +176,19 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(const float *__restrict__
   uint32_t *selbits = dyn + per + 2 * ccap;                     // [per/32]
   const float *srow = scores + (size_t)r * nc_max;
 
-  // ---- A: keys, min / max.  Scores stream from L2 as 16-byte vectors, eight
-  // in flight per thread, where the row's alignment allows it.
+  if (tid == 0) sh.ncand = 0;
+  Binner bin;
+  bin.fixed = hrow != nullptr;
+  bin.fmin = 0.f;
+  bin.scale = 0.f;
+  if (hrow) {
+    // ---- B (precomputed): threshold bin from the row's histogram, then clear it
+    find_threshold_bin<kScoreBins>(sh, k, [&](int bn) { return __ldg(hrow + bn); });
+    cluster_barrier<CS>();  // every CTA has read the row
+    for (int j = rank * NT + tid; j < kScoreBins; j += CS * NT) hrow[j] = 0;
+  }
+
+  // ---- A: keys (16-byte vector loads, eight in flight per thread)
   uint32_t lmin = 0xFFFFFFFFu, lmax = 0u;
   auto take = [&](int j, float f) {
     const uint32_t key = order_key(f);
@@ -143,97 +196,85 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(const float *__restrict__
     lmin = min(lmin, key);
     lmax = max(lmax, key);
   };
-  const float *src = srow + lo;
-  int head = (int)((16 - (reinterpret_cast<uintptr_t>(src) & 15)) & 15) / 4;  // scalars to 16 B
-  head = min(head, len);
-  for (int j = tid; j < head; j += NT) take(j, __ldg(src + j));
-  const int nvec = (len - head) / 4;
-  const float4 *vsrc = reinterpret_cast<const float4 *>(src + head);
-  constexpr int UNR = 8;
-  for (int u0 = 0; u0 < nvec; u0 += NT * UNR) {
-    float4 f[UNR];
+  {
+    const float *src = srow + lo;
+    int head = (int)((16 - (reinterpret_cast<uintptr_t>(src) & 15)) & 15) / 4;
+    head = min(head, len);
+    for (int j = tid; j < head; j += NT) take(j, __ldg(src + j));
+    const int nvec = (len - head) / 4;
+    const float4 *vsrc = reinterpret_cast<const float4 *>(src + head);
+    constexpr int UNR = 8;
+    for (int u0 = 0; u0 < nvec; u0 += NT * UNR) {
+      float4 f[UNR];
 #pragma unroll
-    for (int i = 0; i < UNR; ++i) {
-      const int u = u0 + i * NT + tid;
-      f[i] = u < nvec ? __ldg(vsrc + u) : make_float4(0.f, 0.f, 0.f, 0.f);
-    }
+      for (int i = 0; i < UNR; ++i) {
+        const int u = u0 + i * NT + tid;
+        f[i] = u < nvec ? __ldg(vsrc + u) : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
 #pragma unroll
-    for (int i = 0; i < UNR; ++i) {
-      const int u = u0 + i * NT + tid;
-      if (u < nvec) {
-        const int j = head + 4 * u;
-        take(j, f[i].x);
-        take(j + 1, f[i].y);
-        take(j + 2, f[i].z);
-        take(j + 3, f[i].w);
+      for (int i = 0; i < UNR; ++i) {
+        const int u = u0 + i * NT + tid;
+        if (u < nvec) {
+          const int j = head + 4 * u;
+          take(j, f[i].x);
+          take(j + 1, f[i].y);
+          take(j + 2, f[i].z);
+          take(j + 3, f[i].w);
+        }
       }
     }
+    for (int j = head + 4 * nvec + tid; j < len; j += NT) take(j, __ldg(src + j));
   }
-  for (int j = head + 4 * nvec + tid; j < len; j += NT) take(j, __ldg(src + j));
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    lmin = min(lmin, __shfl_xor_sync(0xffffffffu, lmin, o));
-    lmax = max(lmax, __shfl_xor_sync(0xffffffffu, lmax, o));
-  }
-  if (lane == 0) {
-    sh.red[0][wid] = lmin;
-    sh.red[1][wid] = lmax;
-  }
-  for (int j = tid; j < kTopkBins; j += NT) sh.hist[j] = 0;
-  if (tid == 0) sh.ncand = 0;
-  __syncthreads();
-  if (tid == 0) {
-    uint32_t a = 0xFFFFFFFFu, z = 0u;
-    for (int w = 0; w < NT / 32; ++w) {
-      a = min(a, sh.red[0][w]);
-      z = max(z, sh.red[1][w]);
-    }
-    sh.kmin = a;
-    sh.kmax = z;
-  }
-  cluster_barrier<CS>();
-  uint32_t gmin = 0xFFFFFFFFu, gmax = 0u;
-#pragma unroll
-  for (int c = 0; c < CS; ++c) {
-    const TopkShared *p = peer_ptr<CS>(&sh, c);
-    gmin = min(gmin, p->kmin);
-    gmax = max(gmax, p->kmax);
-  }
-  const float fmin = key_to_float(gmin), fmax = key_to_float(gmax);
-  const float range = __fsub_rn(fmax, fmin);
-  const float scale = (range > 0.f && range <= 3.0e38f) ? __fdiv_rn((float)kTopkBins, range) : 0.f;
 
-  // ---- B: value histogram, the bin b* of the k-th largest key
-  for (int j = tid; j < len; j += NT) atomicAdd(&sh.hist[value_bin(keys[j], fmin, scale)], 1);
-  cluster_barrier<CS>();
-  constexpr int BPT = kTopkBins / NT;  // bins per thread, in descending order
-  int cnt[BPT], mine = 0;
+  if (!hrow) {
+    // ---- B (in-kernel): the row's [min, max], then a value histogram
 #pragma unroll
-  for (int i = 0; i < BPT; ++i) {
-    const int bin = kTopkBins - 1 - (BPT * tid + i);
-    int s = 0;
-#pragma unroll
-    for (int c = 0; c < CS; ++c) s += peer_ptr<CS>(&sh, c)->hist[bin];
-    cnt[i] = s;
-    mine += s;
-  }
-  int total;
-  int above = block_exclusive_scan(mine, sh.scan, &total);
-#pragma unroll
-  for (int i = 0; i < BPT; ++i) {
-    if (above < k && above + cnt[i] >= k) {
-      sh.info[0] = kTopkBins - 1 - (BPT * tid + i);
-      sh.info[1] = above;
-      sh.info[2] = cnt[i];
+    for (int o = 16; o > 0; o >>= 1) {
+      lmin = min(lmin, __shfl_xor_sync(0xffffffffu, lmin, o));
+      lmax = max(lmax, __shfl_xor_sync(0xffffffffu, lmax, o));
     }
-    above += cnt[i];
+    if (lane == 0) {
+      sh.red[0][wid] = lmin;
+      sh.red[1][wid] = lmax;
+    }
+    for (int j = tid; j < kTopkValueBins; j += NT) sh.hist[j] = 0;
+    __syncthreads();
+    if (tid == 0) {
+      uint32_t a = 0xFFFFFFFFu, z = 0u;
+      for (int w = 0; w < NT / 32; ++w) {
+        a = min(a, sh.red[0][w]);
+        z = max(z, sh.red[1][w]);
+      }
+      sh.kmin = a;
+      sh.kmax = z;
+    }
+    cluster_barrier<CS>();
+    uint32_t gmin = 0xFFFFFFFFu, gmax = 0u;
+#pragma unroll
+    for (int c = 0; c < CS; ++c) {
+      const TopkShared *p = peer_ptr<CS>(&sh, c);
+      gmin = min(gmin, p->kmin);
+      gmax = max(gmax, p->kmax);
+    }
+    const float fmin = key_to_float(gmin), fmax = key_to_float(gmax);
+    const float range = __fsub_rn(fmax, fmin);
+    bin.fmin = fmin;
+    bin.scale = (range > 0.f && range <= 3.0e38f) ? __fdiv_rn((float)kTopkValueBins, range) : 0.f;
+    for (int j = tid; j < len; j += NT) atomicAdd(&sh.hist[bin(keys[j])], 1);
+    cluster_barrier<CS>();
+    find_threshold_bin<kTopkValueBins>(sh, k, [&](int bn) {
+      int s = 0;
+#pragma unroll
+      for (int c = 0; c < CS; ++c) s += peer_ptr<CS>(&sh, c)->hist[bn];
+      return s;
+    });
   }
   __syncthreads();
   const int bstar = sh.info[0];
   const int need = k - sh.info[1];  // keys to take from b*
   const int incand = sh.info[2];    // keys in b* over the whole row
   // keys of b*: mode 0 all selected, 1 selected where marked in selbits,
-  // 2 by the radix threshold (pmask, pval), ties by index
+  // 2 by the radix threshold (pmask, pval) with ties by index
   const int mode = (incand == need) ? 0 : (incand <= kTopkRankCap ? 1 : 2);
   uint32_t pmask = 0u, pval = 0u;
   int need_eq = 0;
@@ -243,7 +284,7 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(const float *__restrict__
     // ---- C1: gather every candidate of the cluster, rank this CTA's own
     for (int j = tid; j < len; j += NT) {
       const uint32_t key = keys[j];
-      if (value_bin(key, fmin, scale) == bstar) {
+      if (bin(key) == bstar) {
         const int u = atomicAdd(&sh.ncand, 1);
         cand_key[u] = key;
         cand_pos[u] = j;
@@ -278,30 +319,42 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(const float *__restrict__
     __syncthreads();
   } else if (mode == 2) {
     // ---- C2: radix select among the keys of b* (degenerate distributions)
-    cluster_barrier<CS>();  // peers are done reading the value histogram
+    cluster_barrier<CS>();  // peers are done reading sh.hist
     need_eq = need;
-    for (int pass = 0; pass < 4; ++pass) {
-      const int shift = 24 - 8 * pass;
+    int shift0, npass;
+    if (bin.fixed) {  // the 12 leading bits are b*; digits of bits 19..12, 11..4, 3..0
+      pmask = 0xFFF00000u;
+      pval = (uint32_t)bstar << 20;
+      shift0 = 12;
+      npass = 3;
+    } else {
+      shift0 = 24;
+      npass = 4;
+    }
+    for (int pass = 0; pass < npass; ++pass) {
+      const int shift = shift0 - 8 * pass;
+      const int sh_ = shift < 0 ? 0 : shift;
+      const uint32_t dmask = shift < 0 ? 15u : 255u;  // the last fixed-bin digit has 4 bits
       int *h = sh.hist + 256 * (pass & 1);
       for (int j = tid; j < 256; j += NT) h[j] = 0;
       __syncthreads();
       for (int j0 = 0; j0 < len; j0 += NT) {
         const int j = j0 + tid;
         const uint32_t key = j < len ? keys[j] : 0u;
-        const bool ok = j < len && (key & pmask) == pval && value_bin(key, fmin, scale) == bstar;
+        const bool ok = j < len && (key & pmask) == pval && bin(key) == bstar;
         const unsigned act = __ballot_sync(0xffffffffu, ok);
         if (ok) {
-          const uint32_t bin = (key >> shift) & 255u;
-          const unsigned same = __match_any_sync(act, bin);
-          if (lane == __ffs(same) - 1) atomicAdd(&h[bin], __popc(same));
+          const uint32_t dg = (key >> sh_) & dmask;
+          const unsigned same = __match_any_sync(act, dg);
+          if (lane == __ffs(same) - 1) atomicAdd(&h[dg], __popc(same));
         }
       }
       cluster_barrier<CS>();
       int c2 = 0;
       if (tid < 256) {
-        const int bin = 255 - tid;
+        const int dg = 255 - tid;
 #pragma unroll
-        for (int c = 0; c < CS; ++c) c2 += peer_ptr<CS>(&sh, c)->hist[256 * (pass & 1) + bin];
+        for (int c = 0; c < CS; ++c) c2 += peer_ptr<CS>(&sh, c)->hist[256 * (pass & 1) + dg];
       }
       int tot2;
       const int ab2 = block_exclusive_scan(c2, sh.scan, &tot2);
@@ -312,8 +365,8 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(const float *__restrict__
       }
       __syncthreads();
       need_eq -= sh.info[1];
-      pmask |= 255u << shift;
-      pval |= (uint32_t)sh.info[0] << shift;
+      pmask |= dmask << sh_;
+      pval |= (uint32_t)sh.info[0] << sh_;
       const bool done = (sh.info[2] == need_eq);
       __syncthreads();  // info is read by every thread before the next pass rewrites it
       if (done) {
@@ -330,7 +383,7 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(const float *__restrict__
   // classify: 1 selected, 2 tied at the radix threshold (mode 2), 0 not
   auto classify = [&](int j) -> int {
     const uint32_t key = keys[j];
-    const int bn = value_bin(key, fmin, scale);
+    const int bn = bin(key);
     if (bn != bstar) return bn > bstar ? 1 : 0;
     if (mode == 0) return 1;
     if (mode == 1) return (int)((selbits[j >> 5] >> (j & 31)) & 1u);
@@ -381,7 +434,7 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(const float *__restrict__
     const unsigned me = __ballot_sync(0xffffffffu, cl == 2);
     // tied keys are taken in index order while eq_rank < take_eq
     const int te_here = max(0, min(__popc(me), take_eq - eq_rank));
-    unsigned mt = me;  // the first te_here tied keys of this group
+    unsigned mt = me;  // keep the first te_here tied keys of this group
     for (int d = __popc(me) - te_here; d > 0; --d) mt &= ~(1u << (31 - __clz(mt)));
     const unsigned mall = ms | mt;
     if ((mall >> lane) & 1u) {

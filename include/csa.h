@@ -83,6 +83,15 @@ CSA_API const char *csa_last_error(void);
  * reports an error. */
 CSA_API int csa_check_device_error(void *stream);
 
+/* Per-kernel timing for performance analysis.  While enabled (per host
+ * thread), every entry point records a pair of CUDA events on its stream
+ * around each kernel it launches; this serialises those kernels.
+ * csa_kernel_timing() waits for the last call's events, writes up to
+ * max_kernels durations (ms, in launch order) and returns the number of
+ * kernels that call launched (or a negative status). */
+CSA_API int csa_set_kernel_timing(int enable);
+CSA_API int csa_kernel_timing(float *ms, int max_kernels);
+
 /* ------------------------------------------------------------------------
  * csa_compress -- CSA overlapping compressor (stride 4, 8-token windows).
  *
@@ -146,7 +155,13 @@ CSA_API int hca_compress(const void *x, const int32_t *lens, int B, int n_max, i
  *   scores_out [B][Tq][nc_max] float, optional (NULL: kept in workspace):
  *                            I[t,i] for visible i, -inf for the rest
  *   workspace, ws_bytes      >= csa_index_topk_workspace_size(...), 16-byte
- *                            aligned; may be NULL when that size is 0
+ *                            aligned; may be NULL when that size is 0.  The
+ *                            workspace holds the scores when scores_out is
+ *                            NULL, followed (B*Tq <= 1024) by per-row score
+ *                            histograms of R*4096 int32, which must be zero
+ *                            before the first call with this workspace; every
+ *                            call leaves them zero again.  Two calls that
+ *                            share a workspace must not overlap in time.
  * Inputs must be finite.  Supported: (HI, dI) with HI in [1, 128] and dI in
  * {32, 64, 128}; 1 <= k <= 4096; nc_max <= 327680 (1.31M tokens).
  * ---------------------------------------------------------------------- */

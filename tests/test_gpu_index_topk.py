@@ -172,3 +172,42 @@ def test_invalid_position_raises_device_error():
         csa.check_device_error()
     assert np.all(to_host(idx) == -1)
     csa.check_device_error()  # cleared
+
+
+def test_fused_histogram_path_matches_split_path_and_cleans_workspace():
+    """csa_index_topk (the scoring kernel histograms the scores for the
+    top-k) against csa_index_scores + csa_topk (in-kernel histogram) on the
+    same inputs: identical indices; the shared workspace's histogram part is
+    zero again after every call, so it can be reused."""
+    seed, B, nc, k = 55, 4, 50000, 1024
+    lens = np.array([4 * nc, 4 * nc - 3, 100 * 4, 3], np.int32)  # includes v <= k rows
+    qI = W.normal(seed, "qI", (B, 1, 64, 128), 1.0, "bf16")
+    w = W.normal(seed, "w", (B, 1, 64), 128 ** -0.5, "bf16")
+    kI = W.normal(seed, "kI", (B, nc, 128), 1.0, "bf16")
+    d = [to_dev(a) for a in (qI, w, kI, lens)]
+    ws = csa.index_topk_workspace(B, 1, nc, False)
+    a1 = to_host(csa.csa_index_topk(*d, k, workspace=ws))
+    assert int(ws.view(torch.int32)[-B * 4096:].abs().sum()) == 0
+    a2 = to_host(csa.csa_index_topk(*d, k, workspace=ws))
+    sc = csa.csa_index_scores(*d)
+    b1 = to_host(csa.csa_topk(sc, d[3], k))
+    csa.check_device_error()
+    np.testing.assert_array_equal(a1, a2)
+    np.testing.assert_array_equal(a1, b1)
+    vis = oracle.visible(lens, B, 1, 4).reshape(-1)
+    np.testing.assert_array_equal(a1.reshape(B, k), oracle.select_topk(to_host(sc).reshape(B, -1), vis, k))
+
+
+def test_kernel_timing_hook():
+    nc = 4096
+    qI = W.normal(3, "qI", (1, 1, 64, 128), 1.0, "bf16")
+    w = W.normal(3, "w", (1, 1, 64), 0.1, "bf16")
+    kI = W.normal(3, "kI", (1, nc, 128), 1.0, "bf16")
+    lens = np.array([4 * nc], np.int32)
+    csa.set_kernel_timing(True)
+    try:
+        csa.csa_index_topk(to_dev(qI), to_dev(w), to_dev(kI), to_dev(lens), 64)
+        t = csa.kernel_timing()
+    finally:
+        csa.set_kernel_timing(False)
+    assert len(t) == 2 and all(x > 0 for x in t)
