@@ -141,8 +141,7 @@ def index_topk_workspace_size(B, Tq, nc_max, has_scores_out=False) -> int:
 
 
 def index_topk_workspace(B, Tq, nc_max, has_scores_out=False, device="cuda"):
-    """A zero-filled workspace for csa_index_topk (reusable across calls on
-    one stream: each call leaves its histogram part zero again)."""
+    """A workspace for csa_index_topk (reusable across calls on one stream)."""
     n = index_topk_workspace_size(B, Tq, nc_max, has_scores_out)
     return torch.zeros(max(n, 16), dtype=torch.uint8, device=device)
 

@@ -281,7 +281,7 @@ int launch_index_fma(const void *qI, const void *w, const void *kI, const int32_
 template <int N, int DI>
 int launch_index_tc(const void *qI, const void *w, const void *kI, const int32_t *lens,
                     const int32_t *q_pos, int R, int Tq, int HI, int nc_max, float *scores,
-                    bool fill, int *hist, cudaStream_t st) {
+                    bool fill, cudaStream_t st) {
   const char *what = "csa_index_scores";
   CUtensorMap tmK, tmQ;
   const int B = R / Tq;
@@ -307,22 +307,21 @@ int launch_index_tc(const void *qI, const void *w, const void *kI, const int32_t
   a.R = R;
   a.stages = stages;
   a.fill_invisible = fill ? 1 : 0;
-  a.hist = hist;
   return launch_cluster(kern, 1, (unsigned)num_sms(), csa::kTcThreads, smem, st, what, tmK, tmQ, a);
 }
 
 template <int DI>
 int launch_index_tc_n(const void *qI, const void *w, const void *kI, const int32_t *lens,
                       const int32_t *q_pos, int R, int Tq, int HI, int nc_max, float *scores,
-                      bool fill, int *hist, cudaStream_t st) {
-  if (HI <= 16) return launch_index_tc<16, DI>(qI, w, kI, lens, q_pos, R, Tq, HI, nc_max, scores, fill, hist, st);
-  if (HI <= 32) return launch_index_tc<32, DI>(qI, w, kI, lens, q_pos, R, Tq, HI, nc_max, scores, fill, hist, st);
-  if (HI <= 64) return launch_index_tc<64, DI>(qI, w, kI, lens, q_pos, R, Tq, HI, nc_max, scores, fill, hist, st);
-  return launch_index_tc<128, DI>(qI, w, kI, lens, q_pos, R, Tq, HI, nc_max, scores, fill, hist, st);
+                      bool fill, cudaStream_t st) {
+  if (HI <= 16) return launch_index_tc<16, DI>(qI, w, kI, lens, q_pos, R, Tq, HI, nc_max, scores, fill, st);
+  if (HI <= 32) return launch_index_tc<32, DI>(qI, w, kI, lens, q_pos, R, Tq, HI, nc_max, scores, fill, st);
+  if (HI <= 64) return launch_index_tc<64, DI>(qI, w, kI, lens, q_pos, R, Tq, HI, nc_max, scores, fill, st);
+  return launch_index_tc<128, DI>(qI, w, kI, lens, q_pos, R, Tq, HI, nc_max, scores, fill, st);
 }
 
 template <int CS>
-int launch_topk(const float *scores, int *hist, const int32_t *lens, const int32_t *q_pos, int R,
+int launch_topk(const float *scores, const int32_t *lens, const int32_t *q_pos, int R,
                 int Tq, int nc_max, int k, int32_t *idx_out, cudaStream_t st) {
   const int per = (nc_max + CS - 1) / CS;
   const size_t smem = csa::topk_dyn_bytes(per > 0 ? per : 1);
@@ -330,7 +329,7 @@ int launch_topk(const float *scores, int *hist, const int32_t *lens, const int32
   int rc = ensure_smem(kern, smem, "csa_index_topk");
   if (rc) return rc;
   return launch_cluster(kern, CS, (unsigned)CS * R, csa::kTopkThreads, smem, st,
-                        "csa_index_topk (select)", scores, hist, lens, q_pos, Tq, nc_max, k, idx_out);
+                        "csa_index_topk (select)", scores, lens, q_pos, Tq, nc_max, k, idx_out);
 }
 
 // ---------------------------------------------------------------------------
@@ -498,11 +497,9 @@ int hca_compress(const void *x, const int32_t *lens, int B, int n_max, int d, in
 }
 
 size_t csa_index_topk_workspace_size(int B, int Tq, int nc_max, int has_scores_out) {
-  if (B <= 0 || Tq <= 0 || nc_max <= 0) return 0;
-  const long R = (long)B * Tq;
-  size_t bytes = (((size_t)(has_scores_out ? 0 : sizeof(float) * (size_t)R * nc_max)) + 255) & ~(size_t)255;
-  if (R <= 1024) bytes += sizeof(int) * (size_t)R * csa::kScoreBins;  // zero-filled histograms
-  return bytes;
+  if (B <= 0 || Tq <= 0 || nc_max <= 0 || has_scores_out) return 0;
+  const size_t bytes = sizeof(float) * (size_t)B * Tq * nc_max;
+  return (bytes + 255) & ~(size_t)255;
 }
 
 }  // extern "C"
@@ -514,7 +511,7 @@ bool index_uses_tc(csa_dtype dt, int dI) { return dt == CSA_BF16 && (dI == 64 ||
 
 int index_scores_impl(const void *q_idx, const void *w, const void *k_idx, const int32_t *lens,
                       const int32_t *q_pos, int B, int Tq, int HI, int dI, int nc_max,
-                      csa_dtype dt, float *scores, bool fill, int *hist, cudaStream_t st) {
+                      csa_dtype dt, float *scores, bool fill, cudaStream_t st) {
   const int R = B * Tq;
   if (R == 0 || nc_max == 0) return CSA_OK;
   if (R > 65535) return fail(CSA_ERR_UNSUPPORTED, "csa_index_scores: B*Tq=%d > 65535", R);
@@ -522,8 +519,8 @@ int index_scores_impl(const void *q_idx, const void *w, const void *k_idx, const
   if (index_uses_tc(dt, dI)) {
     if ((long)B * nc_max >= (1L << 31) || (long)R * HI >= (1L << 31))
       return fail(CSA_ERR_UNSUPPORTED, "csa_index_scores: tensor too large for 32-bit coordinates");
-    return dI == 64 ? launch_index_tc_n<64>(q_idx, w, k_idx, lens, q_pos, R, Tq, HI, nc_max, scores, fill, hist, st)
-                    : launch_index_tc_n<128>(q_idx, w, k_idx, lens, q_pos, R, Tq, HI, nc_max, scores, fill, hist, st);
+    return dI == 64 ? launch_index_tc_n<64>(q_idx, w, k_idx, lens, q_pos, R, Tq, HI, nc_max, scores, fill, st)
+                    : launch_index_tc_n<128>(q_idx, w, k_idx, lens, q_pos, R, Tq, HI, nc_max, scores, fill, st);
   }
   if (dt == CSA_F32) {
     switch (dI) {
@@ -539,24 +536,16 @@ int index_scores_impl(const void *q_idx, const void *w, const void *k_idx, const
   }
 }
 
-int topk_impl(const float *scores, int *hist, const int32_t *lens, const int32_t *q_pos, int B,
+int topk_impl(const float *scores, const int32_t *lens, const int32_t *q_pos, int B,
               int Tq, int nc_max, int k, int32_t *idx_out, cudaStream_t st) {
   const int R = B * Tq;
   if (R == 0) return CSA_OK;
   switch (topk_cluster_size(nc_max)) {
-    case 1: return launch_topk<1>(scores, hist, lens, q_pos, R, Tq, nc_max, k, idx_out, st);
-    case 2: return launch_topk<2>(scores, hist, lens, q_pos, R, Tq, nc_max, k, idx_out, st);
-    case 4: return launch_topk<4>(scores, hist, lens, q_pos, R, Tq, nc_max, k, idx_out, st);
-    default: return launch_topk<8>(scores, hist, lens, q_pos, R, Tq, nc_max, k, idx_out, st);
+    case 1: return launch_topk<1>(scores, lens, q_pos, R, Tq, nc_max, k, idx_out, st);
+    case 2: return launch_topk<2>(scores, lens, q_pos, R, Tq, nc_max, k, idx_out, st);
+    case 4: return launch_topk<4>(scores, lens, q_pos, R, Tq, nc_max, k, idx_out, st);
+    default: return launch_topk<8>(scores, lens, q_pos, R, Tq, nc_max, k, idx_out, st);
   }
-}
-
-// Rows up to this count get the score histogram built by the scoring kernel.
-constexpr long kHistMaxRows = 1024;
-
-size_t scores_ws_bytes(int B, int Tq, int nc_max, int has_scores_out) {
-  if (has_scores_out) return 0;
-  return ((sizeof(float) * (size_t)B * Tq * nc_max) + 255) & ~(size_t)255;
 }
 
 // shared argument checks of the indexer entry points
@@ -598,7 +587,7 @@ int csa_index_scores(const void *q_idx, const void *w, const void *k_idx, const 
   if (!aligned16(q_idx) || !aligned16(w) || !aligned16(k_idx) || !aligned16(scores_out))
     return fail(CSA_ERR_ALIGN, "%s: tensors must be 16-byte aligned", what);
   return index_scores_impl(q_idx, w, k_idx, lens, q_pos, B, Tq, HI, dI, nc_max, dt, scores_out,
-                           true, nullptr, static_cast<cudaStream_t>(stream));
+                           true, static_cast<cudaStream_t>(stream));
 }
 
 int csa_topk(const float *scores, const int32_t *lens, const int32_t *q_pos, int B, int Tq,
@@ -610,8 +599,7 @@ int csa_topk(const float *scores, const int32_t *lens, const int32_t *q_pos, int
   if ((long)B * Tq == 0) return CSA_OK;
   if (!lens || !idx_out || (nc_max > 0 && !scores)) return fail(CSA_ERR_NULL, "%s: a required pointer is NULL", what);
   if (scores && !aligned16(scores)) return fail(CSA_ERR_ALIGN, "%s: scores must be 16-byte aligned", what);
-  return topk_impl(scores, nullptr, lens, q_pos, B, Tq, nc_max, k, idx_out,
-                   static_cast<cudaStream_t>(stream));
+  return topk_impl(scores, lens, q_pos, B, Tq, nc_max, k, idx_out, static_cast<cudaStream_t>(stream));
 }
 
 int csa_index_topk(const void *q_idx, const void *w, const void *k_idx, const int32_t *lens,
@@ -637,17 +625,10 @@ int csa_index_topk(const void *q_idx, const void *w, const void *k_idx, const in
   if (need > 0 && !aligned16(workspace)) return fail(CSA_ERR_ALIGN, "%s: workspace must be 16-byte aligned", what);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   float *scores = scores_out ? scores_out : static_cast<float *>(workspace);
-  // the scoring kernel histograms the scores for the top-k when the rows are
-  // few enough; the histogram part of the workspace is zero on entry and
-  // the top-k kernel clears it again
-  int *hist = nullptr;
-  if (nc_max > 0 && (long)B * Tq <= kHistMaxRows && index_uses_tc(dt, dI))
-    hist = reinterpret_cast<int *>(static_cast<char *>(workspace) +
-                                   scores_ws_bytes(B, Tq, nc_max, scores_out != nullptr));
   rc = index_scores_impl(q_idx, w, k_idx, lens, q_pos, B, Tq, HI, dI, nc_max, dt, scores,
-                         scores_out != nullptr, hist, st);
+                         scores_out != nullptr, st);
   if (rc) return rc;
-  return topk_impl(scores, hist, lens, q_pos, B, Tq, nc_max, k, idx_out, st);
+  return topk_impl(scores, lens, q_pos, B, Tq, nc_max, k, idx_out, st);
 }
 
 int csa_attend(const void *q, const void *kv_c, const void *kv_tok, int n_tok, const int32_t *idx,

@@ -44,7 +44,6 @@ struct IndexTcArgs {
   int Tq, HI, nc_max, R;
   int stages;              // depth of the key-tile ring
   int fill_invisible;      // also write -inf past each row's visible entries
-  int *hist;               // optional [R][kScoreBins]: += score_bin counts of visible entries
 };
 
 // visible entries of query row r (0 for an invalid row; the error is raised)
@@ -275,15 +274,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       for (int h = 0; h < N; ++h) sc = fmaf(wv[h], fmaxf(__uint_as_float(d[h]), 0.f), sc);
       const int i = wk.j * kTcRows + row;
       if (i < a.nc_max) a.scores[(size_t)cur_r * a.nc_max + i] = i < vis ? sc : -INFINITY;
-      if (a.hist) {
-        // the row's score histogram for the top-k: lanes sharing a bin add
-        // once through their leader (fire-and-forget global reductions)
-        const bool in = i < vis;
-        const int bin = in ? score_bin(order_key(sc)) : -1;
-        const unsigned same = __match_any_sync(0xffffffffu, bin);
-        if (in && lane == __ffs(same) - 1)
-          atomicAdd(a.hist + (size_t)cur_r * kScoreBins + bin, __popc(same));
-      }
+
       ++nt;
     }
     // -inf past each row's visible tiles (rows split over the CTAs)

@@ -9,24 +9,20 @@
 //
 // Design (cluster of CS CTAs per row; no spin waits):
 //  A. each CTA loads a contiguous slice of the row's visible scores into
-//     shared memory as order-preserving u32 keys;
-//  B. a histogram over monotone bins of the keys finds the bin b* holding the
-//     k-th largest key and the count above it, which decides every key
-//     outside b*.  Two binnings:
-//       - precomputed (csa_index_topk): the scoring kernel already added each
-//         visible score to a per-row histogram of the 12 leading order-key
-//         bits; every CTA reads that row, then the cluster clears it again;
-//       - in-kernel (csa_topk on caller scores): the cluster agrees on the
-//         row's [min, max] and histograms 2048 bins that split it evenly by
-//         value (round-to-nearest subtract and multiply are monotone).
-//     Both avoid the hot spots of a leading-8-bit radix digit, which fp32
-//     scores mostly share;
-//  C. the keys inside b* ("candidates") are ranked exactly: every CTA reads
-//     all candidates of the cluster through distributed shared memory and
-//     counts, for each of its own, the candidates that beat it under (score
-//     desc, index asc).  When b* holds too many keys for that (a degenerate
-//     distribution, e.g. all scores equal) an MSB-first radix select over the
-//     remaining key bits takes over, ties resolved by index;
+//     shared memory as order-preserving u32 keys and histograms them by their
+//     12 leading bits (sign, exponent, 3 mantissa bits: monotone bins about
+//     1/8 octave wide);
+//  B. the cluster merges the histograms in two levels through distributed
+//     shared memory -- 64 super-bins first, then the 64 bins of the super-bin
+//     that holds the k-th largest key -- and finds that key's bin b* and the
+//     count above it, which decide every key outside b*;
+//  C. the keys inside b* ("candidates", a few hundred for real score
+//     distributions) are ranked exactly: every CTA reads all candidates of
+//     the cluster and, one warp per own candidate, counts the candidates
+//     that beat it under (score desc, index asc).  When b* holds too many
+//     keys for that (a degenerate distribution, e.g. all scores equal) an
+//     MSB-first radix select over the remaining 20 key bits takes over,
+//     ties resolved by index;
 //  D. warp-contiguous 32-key groups: ballots give each selected key its slot,
 //     per-warp and per-CTA counts (exchanged in the cluster) give the
 //     offsets, and the indices come out in ascending order.
@@ -45,14 +41,13 @@ namespace cg = cooperative_groups;
 constexpr int kTopkThreads = 512;
 constexpr int kTopkSliceCap = 40960;   // keys per CTA held in shared memory
 constexpr int kTopkMaxCluster = 8;
-constexpr int kTopkValueBins = 2048;   // in-kernel value histogram
+constexpr int kTopkSuper = 64;         // super-bins of 64 score bins
 constexpr int kTopkRankCap = 2048;     // candidates of a row ranked directly
 
 struct TopkShared {
-  int hist[kTopkValueBins];  // value histogram, later the radix digit histograms
+  int hist[kScoreBins];      // this CTA's score_bin histogram; later radix digits
+  int super[kTopkSuper];     // this CTA's super-bin counts
   int scan[33];
-  uint32_t red[2][kTopkThreads / 32];
-  uint32_t kmin, kmax;       // this CTA's min / max key
   int info[4];               // [0] bin, [1] count above it, [2] count in it
   int ncand;                 // this CTA's candidates (keys in b*)
   int cta_counts[2];         // this CTA's (selected, tied) counts
@@ -85,55 +80,24 @@ __device__ __forceinline__ P *peer_ptr(P *mine, int rank) {
   }
 }
 
-__device__ __forceinline__ float key_to_float(uint32_t k) {
-  const uint32_t u = (k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k;
-  return __uint_as_float(u);
-}
-
-// Monotone bins of the order keys.
-struct Binner {
-  bool fixed;   // score_bin (12 leading key bits) or value bins over [fmin, fmax]
-  float fmin;   // value bins: lower edge
-  float scale;  // value bins: bins / (fmax - fmin); 0 puts every key in bin 0
-  __device__ __forceinline__ int operator()(uint32_t key) const {
-    if (fixed) return score_bin(key);
-    const float x = __fmul_rn(__fsub_rn(key_to_float(key), fmin), scale);
-    const int b = (int)x;  // x >= 0
-    return b < kTopkValueBins - 1 ? b : kTopkValueBins - 1;
-  }
-};
-
-// Bin b* of the k-th largest key given per-bin counts (descending search;
-// BPT bins per thread).  Writes sh.info = {b*, count above, count in b*}.
-template <int NB, typename CountFn>
-__device__ __forceinline__ void find_threshold_bin(TopkShared &sh, int k, CountFn count_of) {
-  constexpr int BPT = NB / kTopkThreads;
+// Descending search over n <= kTopkThreads buckets whose counts thread t
+// supplies for bucket (n - 1 - t): the bucket holding the need-th largest
+// key.  Writes sh.info = {bucket, count above it, count in it}.
+__device__ __forceinline__ void find_bucket(TopkShared &sh, int n, int need, int cnt) {
   const int tid = threadIdx.x;
-  int cnt[BPT], mine = 0;
-#pragma unroll
-  for (int i = 0; i < BPT; ++i) {
-    cnt[i] = count_of(NB - 1 - (BPT * tid + i));
-    mine += cnt[i];
-  }
   int total;
-  int above = block_exclusive_scan(mine, sh.scan, &total);
-#pragma unroll
-  for (int i = 0; i < BPT; ++i) {
-    if (above < k && above + cnt[i] >= k) {
-      sh.info[0] = NB - 1 - (BPT * tid + i);
-      sh.info[1] = above;
-      sh.info[2] = cnt[i];
-    }
-    above += cnt[i];
+  const int above = block_exclusive_scan(tid < n ? cnt : 0, sh.scan, &total);
+  if (tid < n && above < need && above + cnt >= need) {
+    sh.info[0] = n - 1 - tid;
+    sh.info[1] = above;
+    sh.info[2] = cnt;
   }
   __syncthreads();
 }
 
-// idx_out row r: the k selected visible entries, ascending.  hist != nullptr:
-// per-row score_bin histograms of the visible scores (cleared on the way).
+// idx_out row r: the k selected visible entries, ascending.
 template <int CS>
 __global__ void __launch_bounds__(kTopkThreads) k_topk(const float *__restrict__ scores,
-                                                       int *__restrict__ hist,
                                                        const int32_t *__restrict__ lens,
                                                        const int32_t *__restrict__ q_pos, int Tq,
                                                        int nc_max, int k,
@@ -146,7 +110,6 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(const float *__restrict__
   const int b = r / Tq, tq = r % Tq;
   const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
   int32_t *orow = idx_out + (size_t)r * k;
-  int *hrow = hist ? hist + (size_t)r * kScoreBins : nullptr;
   pdl_wait();
   pdl_launch_dependents();
 
@@ -161,8 +124,6 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(const float *__restrict__
   // fewer visible entries than k: all of them, then -1 padding
   if (v <= k) {
     for (int j = rank * NT + tid; j < k; j += CS * NT) orow[j] = j < v ? j : -1;
-    if (hrow)
-      for (int j = rank * NT + tid; j < kScoreBins; j += CS * NT) hrow[j] = 0;
     return;  // uniform across the cluster: no barrier was entered
   }
 
@@ -176,25 +137,17 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(const float *__restrict__
   uint32_t *selbits = dyn + per + 2 * ccap;                     // [per/32]
   const float *srow = scores + (size_t)r * nc_max;
 
+  for (int j = tid; j < kScoreBins; j += NT) sh.hist[j] = 0;
+  if (tid < kTopkSuper) sh.super[tid] = 0;
   if (tid == 0) sh.ncand = 0;
-  Binner bin;
-  bin.fixed = hrow != nullptr;
-  bin.fmin = 0.f;
-  bin.scale = 0.f;
-  if (hrow) {
-    // ---- B (precomputed): threshold bin from the row's histogram, then clear it
-    find_threshold_bin<kScoreBins>(sh, k, [&](int bn) { return __ldg(hrow + bn); });
-    cluster_barrier<CS>();  // every CTA has read the row
-    for (int j = rank * NT + tid; j < kScoreBins; j += CS * NT) hrow[j] = 0;
-  }
+  __syncthreads();
 
-  // ---- A: keys (16-byte vector loads, eight in flight per thread)
-  uint32_t lmin = 0xFFFFFFFFu, lmax = 0u;
+  // ---- A: keys (16-byte vector loads, eight in flight per thread) and the
+  // local histogram of their 12 leading bits
   auto take = [&](int j, float f) {
     const uint32_t key = order_key(f);
     keys[j] = key;
-    lmin = min(lmin, key);
-    lmax = max(lmax, key);
+    atomicAdd(&sh.hist[score_bin(key)], 1);
   };
   {
     const float *src = srow + lo;
@@ -225,49 +178,37 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(const float *__restrict__
     }
     for (int j = head + 4 * nvec + tid; j < len; j += NT) take(j, __ldg(src + j));
   }
+  __syncthreads();
+  {
+    constexpr int BPT = kScoreBins / NT;  // bins per thread, one super-bin per 8 threads
+    int sum = 0;
+#pragma unroll
+    for (int i = 0; i < BPT; ++i) sum += sh.hist[BPT * tid + i];
+    atomicAdd(&sh.super[(BPT * tid) / (kScoreBins / kTopkSuper)], sum);
+  }
 
-  if (!hrow) {
-    // ---- B (in-kernel): the row's [min, max], then a value histogram
+  // ---- B: merge over the cluster: super-bins, then the bins of one
+  cluster_barrier<CS>();
+  {
+    int c1 = 0;
+    if (tid < kTopkSuper) {
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      lmin = min(lmin, __shfl_xor_sync(0xffffffffu, lmin, o));
-      lmax = max(lmax, __shfl_xor_sync(0xffffffffu, lmax, o));
+      for (int c = 0; c < CS; ++c) c1 += peer_ptr<CS>(&sh, c)->super[kTopkSuper - 1 - tid];
     }
-    if (lane == 0) {
-      sh.red[0][wid] = lmin;
-      sh.red[1][wid] = lmax;
+    find_bucket(sh, kTopkSuper, k, c1);
+    const int sstar = sh.info[0], above_s = sh.info[1];
+    __syncthreads();  // info is rewritten below
+    constexpr int W = kScoreBins / kTopkSuper;
+    int c2 = 0;
+    if (tid < W) {
+#pragma unroll
+      for (int c = 0; c < CS; ++c) c2 += peer_ptr<CS>(&sh, c)->hist[W * sstar + W - 1 - tid];
     }
-    for (int j = tid; j < kTopkValueBins; j += NT) sh.hist[j] = 0;
-    __syncthreads();
+    find_bucket(sh, W, k - above_s, c2);
     if (tid == 0) {
-      uint32_t a = 0xFFFFFFFFu, z = 0u;
-      for (int w = 0; w < NT / 32; ++w) {
-        a = min(a, sh.red[0][w]);
-        z = max(z, sh.red[1][w]);
-      }
-      sh.kmin = a;
-      sh.kmax = z;
+      sh.info[0] += W * sstar;
+      sh.info[1] += above_s;
     }
-    cluster_barrier<CS>();
-    uint32_t gmin = 0xFFFFFFFFu, gmax = 0u;
-#pragma unroll
-    for (int c = 0; c < CS; ++c) {
-      const TopkShared *p = peer_ptr<CS>(&sh, c);
-      gmin = min(gmin, p->kmin);
-      gmax = max(gmax, p->kmax);
-    }
-    const float fmin = key_to_float(gmin), fmax = key_to_float(gmax);
-    const float range = __fsub_rn(fmax, fmin);
-    bin.fmin = fmin;
-    bin.scale = (range > 0.f && range <= 3.0e38f) ? __fdiv_rn((float)kTopkValueBins, range) : 0.f;
-    for (int j = tid; j < len; j += NT) atomicAdd(&sh.hist[bin(keys[j])], 1);
-    cluster_barrier<CS>();
-    find_threshold_bin<kTopkValueBins>(sh, k, [&](int bn) {
-      int s = 0;
-#pragma unroll
-      for (int c = 0; c < CS; ++c) s += peer_ptr<CS>(&sh, c)->hist[bn];
-      return s;
-    });
   }
   __syncthreads();
   const int bstar = sh.info[0];
@@ -284,7 +225,7 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(const float *__restrict__
     // ---- C1: gather every candidate of the cluster, rank this CTA's own
     for (int j = tid; j < len; j += NT) {
       const uint32_t key = keys[j];
-      if (bin(key) == bstar) {
+      if (score_bin(key) == bstar) {
         const int u = atomicAdd(&sh.ncand, 1);
         cand_key[u] = key;
         cand_pos[u] = j;
@@ -305,32 +246,29 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(const float *__restrict__
       off += nc;
     }
     __syncthreads();
-    for (int u = tid; u < sh.ncand; u += NT) {
+    // one warp per own candidate, lanes over all candidates of the row
+    for (int u = wid; u < sh.ncand; u += NT / 32) {
       const int pos = cand_pos[u];
       const uint32_t key = cand_key[u];
       const int gi = lo + pos;
       int beat = 0;
-      for (int m = 0; m < incand; ++m) {
+      for (int m = lane; m < incand; m += 32) {
         const uint32_t km = sh.all_key[m];
         beat += (km > key) || (km == key && sh.all_idx[m] < gi);
       }
-      if (beat < need) atomicOr(&selbits[pos >> 5], 1u << (pos & 31));
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) beat += __shfl_xor_sync(0xffffffffu, beat, o);
+      if (lane == 0 && beat < need) atomicOr(&selbits[pos >> 5], 1u << (pos & 31));
     }
     __syncthreads();
   } else if (mode == 2) {
     // ---- C2: radix select among the keys of b* (degenerate distributions)
     cluster_barrier<CS>();  // peers are done reading sh.hist
     need_eq = need;
-    int shift0, npass;
-    if (bin.fixed) {  // the 12 leading bits are b*; digits of bits 19..12, 11..4, 3..0
-      pmask = 0xFFF00000u;
-      pval = (uint32_t)bstar << 20;
-      shift0 = 12;
-      npass = 3;
-    } else {
-      shift0 = 24;
-      npass = 4;
-    }
+    // the 12 leading bits are b*; digits of bits 19..12, 11..4, 3..0
+    pmask = 0xFFF00000u;
+    pval = (uint32_t)bstar << 20;
+    const int shift0 = 12, npass = 3;
     for (int pass = 0; pass < npass; ++pass) {
       const int shift = shift0 - 8 * pass;
       const int sh_ = shift < 0 ? 0 : shift;
@@ -341,7 +279,7 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(const float *__restrict__
       for (int j0 = 0; j0 < len; j0 += NT) {
         const int j = j0 + tid;
         const uint32_t key = j < len ? keys[j] : 0u;
-        const bool ok = j < len && (key & pmask) == pval && bin(key) == bstar;
+        const bool ok = j < len && (key & pmask) == pval;
         const unsigned act = __ballot_sync(0xffffffffu, ok);
         if (ok) {
           const uint32_t dg = (key >> sh_) & dmask;
@@ -383,7 +321,7 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(const float *__restrict__
   // classify: 1 selected, 2 tied at the radix threshold (mode 2), 0 not
   auto classify = [&](int j) -> int {
     const uint32_t key = keys[j];
-    const int bn = bin(key);
+    const int bn = score_bin(key);
     if (bn != bstar) return bn > bstar ? 1 : 0;
     if (mode == 0) return 1;
     if (mode == 1) return (int)((selbits[j >> 5] >> (j & 31)) & 1u);

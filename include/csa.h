@@ -155,13 +155,8 @@ CSA_API int hca_compress(const void *x, const int32_t *lens, int B, int n_max, i
  *   scores_out [B][Tq][nc_max] float, optional (NULL: kept in workspace):
  *                            I[t,i] for visible i, -inf for the rest
  *   workspace, ws_bytes      >= csa_index_topk_workspace_size(...), 16-byte
- *                            aligned; may be NULL when that size is 0.  The
- *                            workspace holds the scores when scores_out is
- *                            NULL, followed (B*Tq <= 1024) by per-row score
- *                            histograms of R*4096 int32, which must be zero
- *                            before the first call with this workspace; every
- *                            call leaves them zero again.  Two calls that
- *                            share a workspace must not overlap in time.
+ *                            aligned; may be NULL when that size is 0 (it
+ *                            holds the scores when scores_out is NULL)
  * Inputs must be finite.  Supported: (HI, dI) with HI in [1, 128] and dI in
  * {32, 64, 128}; 1 <= k <= 4096; nc_max <= 327680 (1.31M tokens).
  * ---------------------------------------------------------------------- */

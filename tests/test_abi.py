@@ -86,11 +86,9 @@ def test_index_topk_validation(L):
     assert "workspace" in err(L)
     assert idx_call(L, B=0) == OK
     assert idx_call(L, dt=3) == E_DTYPE
-    hist = 2 * 3 * 4096 * 4  # per-row score histograms (rows <= 1024)
     need = L.csa_index_topk_workspace_size(2, 3, 1000, 0)
-    assert need >= 2 * 3 * 1000 * 4 + hist
-    assert L.csa_index_topk_workspace_size(2, 3, 1000, 1) == hist
-    assert L.csa_index_topk_workspace_size(2, 1000, 100, 1) == 0  # many rows: no histograms
+    assert need >= 2 * 3 * 1000 * 4 and need % 256 == 0
+    assert L.csa_index_topk_workspace_size(2, 3, 1000, 1) == 0
     assert L.csa_index_topk_workspace_size(0, 3, 1000, 0) == 0
 
 

@@ -174,20 +174,18 @@ def test_invalid_position_raises_device_error():
     csa.check_device_error()  # cleared
 
 
-def test_fused_histogram_path_matches_split_path_and_cleans_workspace():
-    """csa_index_topk (the scoring kernel histograms the scores for the
-    top-k) against csa_index_scores + csa_topk (in-kernel histogram) on the
-    same inputs: identical indices; the shared workspace's histogram part is
-    zero again after every call, so it can be reused."""
+def test_index_topk_matches_split_calls_and_reuses_workspace():
+    """csa_index_topk against csa_index_scores + csa_topk on the same inputs
+    (identical indices), twice through one workspace, with rows that have
+    fewer visible entries than k."""
     seed, B, nc, k = 55, 4, 50000, 1024
-    lens = np.array([4 * nc, 4 * nc - 3, 100 * 4, 3], np.int32)  # includes v <= k rows
+    lens = np.array([4 * nc, 4 * nc - 3, 100 * 4, 3], np.int32)
     qI = W.normal(seed, "qI", (B, 1, 64, 128), 1.0, "bf16")
     w = W.normal(seed, "w", (B, 1, 64), 128 ** -0.5, "bf16")
     kI = W.normal(seed, "kI", (B, nc, 128), 1.0, "bf16")
     d = [to_dev(a) for a in (qI, w, kI, lens)]
     ws = csa.index_topk_workspace(B, 1, nc, False)
     a1 = to_host(csa.csa_index_topk(*d, k, workspace=ws))
-    assert int(ws.view(torch.int32)[-B * 4096:].abs().sum()) == 0
     a2 = to_host(csa.csa_index_topk(*d, k, workspace=ws))
     sc = csa.csa_index_scores(*d)
     b1 = to_host(csa.csa_topk(sc, d[3], k))
