@@ -332,6 +332,40 @@ int launch_topk(const float *scores, const int32_t *lens, const int32_t *q_pos, 
                         "csa_index_topk (select)", scores, lens, q_pos, Tq, nc_max, k, idx_out);
 }
 
+// Whether this device can co-schedule a 16-CTA cluster of the top-k kernel
+// (a non-portable cluster size; checked once per device).
+bool topk16_supported(int nc_max) {
+  static int cache[64] = {0};  // 0 unknown, 1 yes, 2 no
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) return false;
+  if (cache[dev] == 0) {
+    auto kern = csa::k_topk<16>;
+    const size_t smem = csa::topk_dyn_bytes(csa::kTopkSliceCap);
+    int ok = 2;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess &&
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) == cudaSuccess) {
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(16, 1, 1);
+      cfg.blockDim = dim3(csa::kTopkThreads, 1, 1);
+      cfg.dynamicSmemBytes = smem;
+      cudaLaunchAttribute attr;
+      attr.id = cudaLaunchAttributeClusterDimension;
+      attr.val.clusterDim.x = 16;
+      attr.val.clusterDim.y = 1;
+      attr.val.clusterDim.z = 1;
+      cfg.attrs = &attr;
+      cfg.numAttrs = 1;
+      int n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) == cudaSuccess && n > 0) ok = 1;
+    }
+    cudaGetLastError();
+    cache[dev] = ok;
+  }
+  (void)nc_max;
+  return cache[dev] == 1;
+}
+
 // ---------------------------------------------------------------------------
 // attention
 // ---------------------------------------------------------------------------
@@ -540,6 +574,9 @@ int topk_impl(const float *scores, const int32_t *lens, const int32_t *q_pos, in
               int Tq, int nc_max, int k, int32_t *idx_out, cudaStream_t st) {
   const int R = B * Tq;
   if (R == 0) return CSA_OK;
+  // long rows: a 16-CTA cluster where the device can schedule one
+  if (nc_max > 8 * 16384 && topk16_supported(nc_max))
+    return launch_topk<16>(scores, lens, q_pos, R, Tq, nc_max, k, idx_out, st);
   switch (topk_cluster_size(nc_max)) {
     case 1: return launch_topk<1>(scores, lens, q_pos, R, Tq, nc_max, k, idx_out, st);
     case 2: return launch_topk<2>(scores, lens, q_pos, R, Tq, nc_max, k, idx_out, st);

@@ -55,11 +55,12 @@ struct TopkShared {
   int all_idx[kTopkRankCap];
 };
 
-// Dynamic shared memory of one CTA for slices of up to `per` keys: the keys,
-// the candidates (key and position) and the selection bit mask.
+// Dynamic shared memory of one CTA for slices of up to `per` keys: the keys
+// (plus alignment slack), the candidates (key and position) and two bit
+// masks over the slice (keys above the threshold bin, chosen candidates).
 __host__ __device__ constexpr size_t topk_dyn_bytes(int per) {
-  return 4ull * ((size_t)per + 2 * (size_t)(per < kTopkRankCap ? per : kTopkRankCap) +
-                 ((size_t)per + 31) / 32);
+  return 4ull * ((size_t)per + 4 + 2 * (size_t)(per < kTopkRankCap ? per : kTopkRankCap) +
+                 2 * (((size_t)per + 31) / 32));
 }
 
 template <int CS>
@@ -131,11 +132,16 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(const float *__restrict__
   const int lo = min(v, rank * per), hi = min(v, lo + per);
   const int len = hi - lo;
   const int ccap = per < kTopkRankCap ? per : kTopkRankCap;
-  uint32_t *keys = dyn;                                         // [per]
-  uint32_t *cand_key = dyn + per;                               // [ccap]
-  int *cand_pos = reinterpret_cast<int *>(dyn + per + ccap);    // [ccap]
-  uint32_t *selbits = dyn + per + 2 * ccap;                     // [per/32]
+  const int nwords = (per + 31) / 32;
   const float *srow = scores + (size_t)r * nc_max;
+  // the slice start's misalignment to 16 B, mirrored in the key array so that
+  // vector loads and vector stores line up
+  const int head0 = (int)((16 - (reinterpret_cast<uintptr_t>(srow + lo) & 15)) & 15) / 4;
+  uint32_t *keys = dyn + ((4 - head0) & 3);                     // [per], keys+head0 16 B aligned
+  uint32_t *cand_key = dyn + per + 4;                           // [ccap]
+  int *cand_pos = reinterpret_cast<int *>(dyn + per + 4 + ccap);  // [ccap]
+  uint32_t *selbits = dyn + per + 4 + 2 * ccap;                 // [nwords] chosen candidates
+  uint32_t *abovebits = selbits + nwords;                       // [nwords] keys above b*
 
   for (int j = tid; j < kScoreBins; j += NT) sh.hist[j] = 0;
   if (tid < kTopkSuper) sh.super[tid] = 0;
@@ -151,11 +157,11 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(const float *__restrict__
   };
   {
     const float *src = srow + lo;
-    int head = (int)((16 - (reinterpret_cast<uintptr_t>(src) & 15)) & 15) / 4;
-    head = min(head, len);
+    const int head = min(head0, len);
     for (int j = tid; j < head; j += NT) take(j, __ldg(src + j));
     const int nvec = (len - head) / 4;
     const float4 *vsrc = reinterpret_cast<const float4 *>(src + head);
+    uint4 *vkeys = reinterpret_cast<uint4 *>(keys + head);
     constexpr int UNR = 8;
     for (int u0 = 0; u0 < nvec; u0 += NT * UNR) {
       float4 f[UNR];
@@ -168,11 +174,13 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(const float *__restrict__
       for (int i = 0; i < UNR; ++i) {
         const int u = u0 + i * NT + tid;
         if (u < nvec) {
-          const int j = head + 4 * u;
-          take(j, f[i].x);
-          take(j + 1, f[i].y);
-          take(j + 2, f[i].z);
-          take(j + 3, f[i].w);
+          const uint4 kv = make_uint4(order_key(f[i].x), order_key(f[i].y), order_key(f[i].z),
+                                      order_key(f[i].w));
+          vkeys[u] = kv;
+          atomicAdd(&sh.hist[score_bin(kv.x)], 1);
+          atomicAdd(&sh.hist[score_bin(kv.y)], 1);
+          atomicAdd(&sh.hist[score_bin(kv.z)], 1);
+          atomicAdd(&sh.hist[score_bin(kv.w)], 1);
         }
       }
     }
@@ -221,17 +229,39 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(const float *__restrict__
   int need_eq = 0;
   bool all_eq = false;
 
-  if (mode == 1) {
-    // ---- C1: gather every candidate of the cluster, rank this CTA's own
-    for (int j = tid; j < len; j += NT) {
-      const uint32_t key = keys[j];
-      if (score_bin(key) == bstar) {
-        const int u = atomicAdd(&sh.ncand, 1);
-        cand_key[u] = key;
-        cand_pos[u] = j;
+  // warp w owns the contiguous chunk [w*cw, (w+1)*cw) of the slice, walked in
+  // groups of 32 consecutive keys (group g = bit-mask word g)
+  constexpr int NW = NT / 32;
+  const int cw = ((len + NW - 1) / NW + 31) & ~31;
+  const int w0 = min(len, wid * cw), w1 = min(len, w0 + cw);
+  const unsigned lt = (1u << lane) - 1u;
+
+  if (mode != 2) {
+    // ---- C: one pass: keys above b* (and all of b* in mode 0) into
+    // abovebits; in mode 1 the keys of b* into the candidate list
+    for (int g = w0; g < w1; g += 32) {
+      const int j = g + lane;
+      const int bn = j < w1 ? score_bin(keys[j]) : -1;
+      const unsigned ma = __ballot_sync(0xffffffffu, mode == 0 ? bn >= bstar : bn > bstar);
+      const unsigned mc = __ballot_sync(0xffffffffu, mode == 1 && bn == bstar);
+      if (lane == 0) {
+        abovebits[g >> 5] = ma;
+        selbits[g >> 5] = 0u;
+      }
+      if (mc) {
+        int base = 0;
+        if (lane == 0) base = atomicAdd(&sh.ncand, __popc(mc));
+        base = __shfl_sync(0xffffffffu, base, 0);
+        if ((mc >> lane) & 1u) {
+          const int u = base + __popc(mc & lt);
+          cand_key[u] = keys[j];
+          cand_pos[u] = j;
+        }
       }
     }
-    for (int j = tid; j < (len + 31) / 32; j += NT) selbits[j] = 0u;
+  }
+  if (mode == 1) {
+    // ---- C1: gather every candidate of the cluster, rank this CTA's own
     cluster_barrier<CS>();
     int off = 0;
     for (int c = 0; c < CS; ++c) {
@@ -314,32 +344,27 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(const float *__restrict__
     }
   }
 
-  // ---- D: count, exchange offsets, write in index order.  Warp w owns the
-  // contiguous chunk [w*cw, (w+1)*cw) of the slice and walks it in groups of
-  // 32 consecutive keys (lane = key: conflict-free shared-memory reads);
-  // positions come from ballots within a group and scans across warps.
-  // classify: 1 selected, 2 tied at the radix threshold (mode 2), 0 not
+  // ---- D: count, exchange offsets, write in index order
+  // classify (mode 2): 1 selected, 2 tied at the radix threshold, 0 not
   auto classify = [&](int j) -> int {
     const uint32_t key = keys[j];
     const int bn = score_bin(key);
     if (bn != bstar) return bn > bstar ? 1 : 0;
-    if (mode == 0) return 1;
-    if (mode == 1) return (int)((selbits[j >> 5] >> (j & 31)) & 1u);
     const uint32_t km = key & pmask;
     if (km > pval) return 1;
     if (km == pval) return all_eq ? 1 : 2;
     return 0;
   };
-  constexpr int NW = NT / 32;
-  const int cw = ((len + NW - 1) / NW + 31) & ~31;
-  const int w0 = min(len, wid * cw), w1 = min(len, w0 + cw);
-  const unsigned lt = (1u << lane) - 1u;
   int n_sel = 0, n_eq = 0;  // warp totals (identical in every lane)
-  for (int g = w0; g < w1; g += 32) {
-    const int j = g + lane;
-    const int cl = j < w1 ? classify(j) : 0;
-    n_sel += __popc(__ballot_sync(0xffffffffu, cl == 1));
-    n_eq += __popc(__ballot_sync(0xffffffffu, cl == 2));
+  if (mode != 2) {
+    for (int g = w0; g < w1; g += 32) n_sel += __popc(abovebits[g >> 5] | selbits[g >> 5]);
+  } else {
+    for (int g = w0; g < w1; g += 32) {
+      const int j = g + lane;
+      const int cl = j < w1 ? classify(j) : 0;
+      n_sel += __popc(__ballot_sync(0xffffffffu, cl == 1));
+      n_eq += __popc(__ballot_sync(0xffffffffu, cl == 2));
+    }
   }
   int cta_sel, cta_eq;
   const int sel_before = block_exclusive_scan(lane == 0 ? n_sel : 0, sh.scan, &cta_sel);
@@ -366,23 +391,28 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(const float *__restrict__
   int pos = off + wsel + max(0, min(weq, take_eq));
   int eq_rank = weq;
   for (int g = w0; g < w1; g += 32) {
-    const int j = g + lane;
-    const int cl = j < w1 ? classify(j) : 0;
-    const unsigned ms = __ballot_sync(0xffffffffu, cl == 1);
-    const unsigned me = __ballot_sync(0xffffffffu, cl == 2);
-    // tied keys are taken in index order while eq_rank < take_eq
-    const int te_here = max(0, min(__popc(me), take_eq - eq_rank));
-    unsigned mt = me;  // keep the first te_here tied keys of this group
-    for (int d = __popc(me) - te_here; d > 0; --d) mt &= ~(1u << (31 - __clz(mt)));
-    const unsigned mall = ms | mt;
+    unsigned mall;
+    if (mode != 2) {
+      mall = abovebits[g >> 5] | selbits[g >> 5];
+    } else {
+      const int j = g + lane;
+      const int cl = j < w1 ? classify(j) : 0;
+      const unsigned ms = __ballot_sync(0xffffffffu, cl == 1);
+      const unsigned me = __ballot_sync(0xffffffffu, cl == 2);
+      // tied keys are taken in index order while eq_rank < take_eq
+      const int te_here = max(0, min(__popc(me), take_eq - eq_rank));
+      unsigned mt = me;  // keep the first te_here tied keys of this group
+      for (int d = __popc(me) - te_here; d > 0; --d) mt &= ~(1u << (31 - __clz(mt)));
+      mall = ms | mt;
+      eq_rank += __popc(me);
+    }
     if ((mall >> lane) & 1u) {
       const int p = pos + __popc(mall & lt);
       // (p < k always holds: exactly k keys are selected; the guard keeps a
       // miscount from ever writing outside the row)
-      if (p < k) orow[p] = lo + j;
+      if (p < k) orow[p] = lo + g + lane;
     }
     pos += __popc(mall);
-    eq_rank += __popc(me);
   }
   cluster_barrier<CS>();  // peers may still read this CTA's shared memory
 }
