@@ -51,6 +51,7 @@ struct TopkShared {
   int info[4];               // [0] bin, [1] count above it, [2] count in it
   int ncand;                 // this CTA's candidates (keys in b*)
   int cta_counts[2];         // this CTA's (selected, tied) counts
+  int peer_nc[16];           // candidates of each CTA of the cluster
   uint32_t all_key[kTopkRankCap];
   int all_idx[kTopkRankCap];
 };
@@ -263,17 +264,20 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(const float *__restrict__
   if (mode == 1) {
     // ---- C1: gather every candidate of the cluster, rank this CTA's own
     cluster_barrier<CS>();
-    int off = 0;
-    for (int c = 0; c < CS; ++c) {
-      const int nc = peer_ptr<CS>(&sh, c)->ncand;
-      const int *pc = peer_ptr<CS>(cand_pos, c);
-      const uint32_t *pk = peer_ptr<CS>(cand_key, c);
-      const int plo = min(v, c * per);
-      for (int u = tid; u < nc; u += NT) {
-        sh.all_key[off + u] = pk[u];
-        sh.all_idx[off + u] = plo + pc[u];
-      }
-      off += nc;
+    // every peer's candidate count in parallel, then all candidates at once
+    if (tid < CS) sh.peer_nc[tid] = peer_ptr<CS>(&sh, tid)->ncand;
+    __syncthreads();
+    int coff[CS + 1];
+    coff[0] = 0;
+#pragma unroll
+    for (int c = 0; c < CS; ++c) coff[c + 1] = coff[c] + sh.peer_nc[c];
+    for (int m = tid; m < coff[CS]; m += NT) {
+      int c = 0;
+#pragma unroll
+      for (int cc = 1; cc < CS; ++cc) c += m >= coff[cc];
+      const int u = m - coff[c];
+      sh.all_key[m] = peer_ptr<CS>(cand_key, c)[u];
+      sh.all_idx[m] = min(v, c * per) + peer_ptr<CS>(cand_pos, c)[u];
     }
     __syncthreads();
     // one warp per own candidate, lanes over all candidates of the row
