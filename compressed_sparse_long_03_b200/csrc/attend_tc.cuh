@@ -47,7 +47,7 @@ __global__ void __launch_bounds__(kAtThreads, 1) k_attend_tc(AttendArgs a) {
   extern __shared__ uint8_t smem_raw[];
   __shared__ uint32_t tmem_holder;
   __shared__ uint64_t bar_s, bar_o;
-  __shared__ int kvalid[kAtMaxTile];
+  __shared__ int kvalid[kAtMaxTile / 32];  // validity bits, one word per 32 keys
   __shared__ const __nv_bfloat16 *rowp[kAtMaxTile];
   __shared__ float pm[128], pl[128];
   __shared__ float mw[136], minv[128];  // merge weights [head][rank], 1 / sum
@@ -147,7 +147,9 @@ __global__ void __launch_bounds__(kAtThreads, 1) k_attend_tc(AttendArgs a) {
         }
       }
       rowp[j] = row;
-      kvalid[j] = row != nullptr;
+      // a warp covers 32 consecutive keys: one validity word per 32
+      const unsigned vm = __ballot_sync(0xffffffffu, row != nullptr);
+      if ((tid & 31) == 0) kvalid[j >> 5] = (int)vm;
     }
     __syncthreads();
     for (int u = tid; u < nchunk * 32 * 16; u += kAtThreads) {
@@ -185,26 +187,28 @@ __global__ void __launch_bounds__(kAtThreads, 1) k_attend_tc(AttendArgs a) {
       tmem_ld16(tS + lane_off + 32 * c, sv);
       tmem_ld16(tS + lane_off + 32 * c + 16, sv + 16);
       tmem_wait_ld_regs<32>(sv);
+      const uint32_t vm = (uint32_t)kvalid[c];
 #pragma unroll
       for (int jj = 0; jj < 32; ++jj)
-        if (kvalid[32 * c + jj]) mt = fmaxf(mt, __uint_as_float(sv[jj]) * a.scale_log2);
+        if ((vm >> jj) & 1u) mt = fmaxf(mt, __uint_as_float(sv[jj]) * a.scale_log2);
     }
     const float m_new = fmaxf(m_run, mt);
-    const float alpha = (m_new == -INFINITY) ? 1.f : exp2f(m_run - m_new);
+    const float alpha = (m_new == -INFINITY) ? 1.f : ex2(m_run - m_new);
     float lsum = 0.f;
     for (int c = 0; c < nchunk; ++c) {
       uint32_t sv[32];
       tmem_ld16(tS + lane_off + 32 * c, sv);
       tmem_ld16(tS + lane_off + 32 * c + 16, sv + 16);
       tmem_wait_ld_regs<32>(sv);
+      const uint32_t vm = (uint32_t)kvalid[c];
 #pragma unroll
       for (int g = 0; g < 4; ++g) {  // 8 keys -> one 16-byte chunk of P
         uint32_t pk[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const int j0 = 8 * g + 2 * e;
-          const float p0v = kvalid[32 * c + j0] ? exp2f(__uint_as_float(sv[j0]) * a.scale_log2 - m_new) : 0.f;
-          const float p1v = kvalid[32 * c + j0 + 1] ? exp2f(__uint_as_float(sv[j0 + 1]) * a.scale_log2 - m_new) : 0.f;
+          const float p0v = ((vm >> j0) & 1u) ? ex2(__uint_as_float(sv[j0]) * a.scale_log2 - m_new) : 0.f;
+          const float p1v = ((vm >> (j0 + 1)) & 1u) ? ex2(__uint_as_float(sv[j0 + 1]) * a.scale_log2 - m_new) : 0.f;
           lsum += p0v + p1v;
           __nv_bfloat162 pr = __floats2bfloat162_rn(p0v, p1v);
           pk[e] = *reinterpret_cast<uint32_t *>(&pr);
@@ -276,7 +280,7 @@ __global__ void __launch_bounds__(kAtThreads, 1) k_attend_tc(AttendArgs a) {
 #pragma unroll
     for (int c = 0; c < CS; ++c) {
       const float mc = att_peer<CS>(pm, c)[h];
-      const float wgt = (mc == -INFINITY) ? 0.f : exp2f(mc - M);
+      const float wgt = (mc == -INFINITY) ? 0.f : ex2(mc - M);
       Ls = fmaf(att_peer<CS>(pl, c)[h], wgt, Ls);
       mw[tid * CS + c] = wgt;
     }

@@ -7,25 +7,29 @@
 // the order (score desc, index asc): ties go to the lower index; -0.0 ranks
 // as +0.0; every visible entry when fewer than k.
 //
-// Design (cluster of CS CTAs per row; no spin waits):
+// Design (cluster of CS CTAs per row; three cluster barriers; no spin waits):
 //  A. each CTA loads a contiguous slice of the row's visible scores into
 //     shared memory as order-preserving u32 keys and histograms them by their
 //     12 leading bits (sign, exponent, 3 mantissa bits: monotone bins about
-//     1/8 octave wide);
+//     1/8 octave wide);                                         [barrier 1]
 //  B. the cluster merges the histograms in two levels through distributed
-//     shared memory -- 64 super-bins first, then the 64 bins of the super-bin
-//     that holds the k-th largest key -- and finds that key's bin b* and the
-//     count above it, which decide every key outside b*;
-//  C. the keys inside b* ("candidates", a few hundred for real score
-//     distributions) are ranked exactly: every CTA reads all candidates of
-//     the cluster and, one warp per own candidate, counts the candidates
-//     that beat it under (score desc, index asc).  When b* holds too many
-//     keys for that (a degenerate distribution, e.g. all scores equal) an
-//     MSB-first radix select over the remaining 20 key bits takes over,
-//     ties resolved by index;
-//  D. warp-contiguous 32-key groups: ballots give each selected key its slot,
-//     per-warp and per-CTA counts (exchanged in the cluster) give the
-//     offsets, and the indices come out in ascending order.
+//     shared memory -- 64 super-bins, then the 64 bins of the super-bin that
+//     holds the k-th largest key -- giving that key's bin b* and the count
+//     above it: every key outside b* is decided;
+//  C. one pass over the slice marks the keys above b* in a bit mask (one
+//     word per 32 keys) and collects the keys inside b* ("candidates", a few
+//     hundred for real score distributions);                   [barrier 2]
+//     every CTA then gathers all candidates of the cluster and resolves them
+//     locally, identically: an 8-bit radix step on key bits 19..12 finds the
+//     threshold sub-bin, and inside it candidates are ranked pairwise under
+//     (score desc, index asc).  So every CTA knows how many keys each CTA of
+//     the cluster selects;
+//  D. the output offsets follow from those counts and from per-warp bit
+//     counts, and each CTA writes its selected indices in ascending order
+//     straight from the bit masks.                        [barrier 3: exit]
+// When b* holds more candidates than fit (a degenerate distribution, e.g.
+// all scores equal) an MSB-first radix select over the keys of b* with
+// cluster-wide digit histograms takes over, ties resolved by index.
 // All decisions are integer comparisons on the same keys in every CTA, so
 // the result is bit-exact and independent of the launch configuration.
 #pragma once
@@ -38,11 +42,11 @@ namespace csa {
 
 namespace cg = cooperative_groups;
 
-constexpr int kTopkThreads = 512;
+constexpr int kTopkThreads = 1024;
 constexpr int kTopkSliceCap = 40960;   // keys per CTA held in shared memory
-constexpr int kTopkMaxCluster = 8;
+constexpr int kTopkMaxCluster = 8;     // portable; 16 where the device allows
 constexpr int kTopkSuper = 64;         // super-bins of 64 score bins
-constexpr int kTopkRankCap = 2048;     // candidates of a row ranked directly
+constexpr int kTopkRankCap = 2048;     // candidates of a row resolved locally
 
 struct TopkShared {
   int hist[kScoreBins];      // this CTA's score_bin histogram; later radix digits
@@ -50,10 +54,12 @@ struct TopkShared {
   int scan[33];
   int info[4];               // [0] bin, [1] count above it, [2] count in it
   int ncand;                 // this CTA's candidates (keys in b*)
-  int cta_counts[2];         // this CTA's (selected, tied) counts
-  int peer_nc[16];           // candidates of each CTA of the cluster
+  int above;                 // this CTA's keys above b* (all of b* in mode 0)
+  int cta_counts[2];         // legacy path: this CTA's (selected, tied) counts
+  int peer_nc[16], peer_above[16], peer_sel[16];
   uint32_t all_key[kTopkRankCap];
   int all_idx[kTopkRankCap];
+  unsigned char all_cta[kTopkRankCap];
 };
 
 // Dynamic shared memory of one CTA for slices of up to `per` keys: the keys
@@ -82,7 +88,7 @@ __device__ __forceinline__ P *peer_ptr(P *mine, int rank) {
   }
 }
 
-// Descending search over n <= kTopkThreads buckets whose counts thread t
+// Descending search over n <= blockDim buckets whose counts thread t
 // supplies for bucket (n - 1 - t): the bucket holding the need-th largest
 // key.  Writes sh.info = {bucket, count above it, count in it}.
 __device__ __forceinline__ void find_bucket(TopkShared &sh, int n, int need, int cnt) {
@@ -106,11 +112,12 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(const float *__restrict__
                                                        int32_t *__restrict__ idx_out) {
   extern __shared__ uint32_t dyn[];
   __shared__ TopkShared sh;
-  constexpr int NT = kTopkThreads;
+  constexpr int NT = kTopkThreads, NW = NT / 32;
   const int rank = (CS > 1) ? (int)cg::this_cluster().block_rank() : 0;
   const int r = blockIdx.x / CS;  // clusters tile the grid along x
   const int b = r / Tq, tq = r % Tq;
   const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+  const unsigned lt = (1u << lane) - 1u;
   int32_t *orow = idx_out + (size_t)r * k;
   pdl_wait();
   pdl_launch_dependents();
@@ -138,27 +145,31 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(const float *__restrict__
   // the slice start's misalignment to 16 B, mirrored in the key array so that
   // vector loads and vector stores line up
   const int head0 = (int)((16 - (reinterpret_cast<uintptr_t>(srow + lo) & 15)) & 15) / 4;
-  uint32_t *keys = dyn + ((4 - head0) & 3);                     // [per], keys+head0 16 B aligned
-  uint32_t *cand_key = dyn + per + 4;                           // [ccap]
+  uint32_t *keys = dyn + ((4 - head0) & 3);                       // [per], keys+head0 16 B aligned
+  uint32_t *cand_key = dyn + per + 4;                             // [ccap]
   int *cand_pos = reinterpret_cast<int *>(dyn + per + 4 + ccap);  // [ccap]
-  uint32_t *selbits = dyn + per + 4 + 2 * ccap;                 // [nwords] chosen candidates
-  uint32_t *abovebits = selbits + nwords;                       // [nwords] keys above b*
+  uint32_t *selbits = dyn + per + 4 + 2 * ccap;                   // [nwords] chosen candidates
+  uint32_t *abovebits = selbits + nwords;                         // [nwords] decided above b*
 
   for (int j = tid; j < kScoreBins; j += NT) sh.hist[j] = 0;
   if (tid < kTopkSuper) sh.super[tid] = 0;
-  if (tid == 0) sh.ncand = 0;
+  if (tid == 0) {
+    sh.ncand = 0;
+    sh.above = 0;
+  }
+  if (tid < 16) sh.peer_sel[tid] = 0;
   __syncthreads();
 
   // ---- A: keys (16-byte vector loads, eight in flight per thread) and the
   // local histogram of their 12 leading bits
-  auto take = [&](int j, float f) {
-    const uint32_t key = order_key(f);
-    keys[j] = key;
-    atomicAdd(&sh.hist[score_bin(key)], 1);
-  };
   {
     const float *src = srow + lo;
     const int head = min(head0, len);
+    auto take = [&](int j, float f) {
+      const uint32_t key = order_key(f);
+      keys[j] = key;
+      atomicAdd(&sh.hist[score_bin(key)], 1);
+    };
     for (int j = tid; j < head; j += NT) take(j, __ldg(src + j));
     const int nvec = (len - head) / 4;
     const float4 *vsrc = reinterpret_cast<const float4 *>(src + head);
@@ -189,7 +200,7 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(const float *__restrict__
   }
   __syncthreads();
   {
-    constexpr int BPT = kScoreBins / NT;  // bins per thread, one super-bin per 8 threads
+    constexpr int BPT = kScoreBins / NT;  // bins per thread
     int sum = 0;
 #pragma unroll
     for (int i = 0; i < BPT; ++i) sum += sh.hist[BPT * tid + i];
@@ -197,7 +208,7 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(const float *__restrict__
   }
 
   // ---- B: merge over the cluster: super-bins, then the bins of one
-  cluster_barrier<CS>();
+  cluster_barrier<CS>();  // [1]
   {
     int c1 = 0;
     if (tid < kTopkSuper) {
@@ -207,15 +218,15 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(const float *__restrict__
     find_bucket(sh, kTopkSuper, k, c1);
     const int sstar = sh.info[0], above_s = sh.info[1];
     __syncthreads();  // info is rewritten below
-    constexpr int W = kScoreBins / kTopkSuper;
+    constexpr int Wb = kScoreBins / kTopkSuper;
     int c2 = 0;
-    if (tid < W) {
+    if (tid < Wb) {
 #pragma unroll
-      for (int c = 0; c < CS; ++c) c2 += peer_ptr<CS>(&sh, c)->hist[W * sstar + W - 1 - tid];
+      for (int c = 0; c < CS; ++c) c2 += peer_ptr<CS>(&sh, c)->hist[Wb * sstar + Wb - 1 - tid];
     }
-    find_bucket(sh, W, k - above_s, c2);
+    find_bucket(sh, Wb, k - above_s, c2);
     if (tid == 0) {
-      sh.info[0] += W * sstar;
+      sh.info[0] += Wb * sstar;
       sh.info[1] += above_s;
     }
   }
@@ -223,23 +234,18 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(const float *__restrict__
   const int bstar = sh.info[0];
   const int need = k - sh.info[1];  // keys to take from b*
   const int incand = sh.info[2];    // keys in b* over the whole row
-  // keys of b*: mode 0 all selected, 1 selected where marked in selbits,
-  // 2 by the radix threshold (pmask, pval) with ties by index
+  // keys of b*: mode 0 all selected; 1 resolved locally from the gathered
+  // candidates; 2 the cluster-wide radix fallback
   const int mode = (incand == need) ? 0 : (incand <= kTopkRankCap ? 1 : 2);
-  uint32_t pmask = 0u, pval = 0u;
-  int need_eq = 0;
-  bool all_eq = false;
 
   // warp w owns the contiguous chunk [w*cw, (w+1)*cw) of the slice, walked in
-  // groups of 32 consecutive keys (group g = bit-mask word g)
-  constexpr int NW = NT / 32;
+  // groups of 32 consecutive keys (group g = bit-mask word g/32)
   const int cw = ((len + NW - 1) / NW + 31) & ~31;
   const int w0 = min(len, wid * cw), w1 = min(len, w0 + cw);
-  const unsigned lt = (1u << lane) - 1u;
 
   if (mode != 2) {
-    // ---- C: one pass: keys above b* (and all of b* in mode 0) into
-    // abovebits; in mode 1 the keys of b* into the candidate list
+    // ---- C: decided keys into abovebits, candidates into the list
+    int my_above = 0;
     for (int g = w0; g < w1; g += 32) {
       const int j = g + lane;
       const int bn = j < w1 ? score_bin(keys[j]) : -1;
@@ -249,6 +255,7 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(const float *__restrict__
         abovebits[g >> 5] = ma;
         selbits[g >> 5] = 0u;
       }
+      my_above += __popc(ma);
       if (mc) {
         int base = 0;
         if (lane == 0) base = atomicAdd(&sh.ncand, __popc(mc));
@@ -260,96 +267,145 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(const float *__restrict__
         }
       }
     }
-  }
-  if (mode == 1) {
-    // ---- C1: gather every candidate of the cluster, rank this CTA's own
-    cluster_barrier<CS>();
-    // every peer's candidate count in parallel, then all candidates at once
-    if (tid < CS) sh.peer_nc[tid] = peer_ptr<CS>(&sh, tid)->ncand;
-    __syncthreads();
-    int coff[CS + 1];
-    coff[0] = 0;
-#pragma unroll
-    for (int c = 0; c < CS; ++c) coff[c + 1] = coff[c] + sh.peer_nc[c];
-    for (int m = tid; m < coff[CS]; m += NT) {
-      int c = 0;
-#pragma unroll
-      for (int cc = 1; cc < CS; ++cc) c += m >= coff[cc];
-      const int u = m - coff[c];
-      sh.all_key[m] = peer_ptr<CS>(cand_key, c)[u];
-      sh.all_idx[m] = min(v, c * per) + peer_ptr<CS>(cand_pos, c)[u];
+    if (lane == 0 && my_above) atomicAdd(&sh.above, my_above);
+    cluster_barrier<CS>();  // [2]
+    if (tid < CS) {
+      const TopkShared *p = peer_ptr<CS>(&sh, tid);
+      sh.peer_nc[tid] = p->ncand;
+      sh.peer_above[tid] = p->above;
     }
     __syncthreads();
-    // one warp per own candidate, lanes over all candidates of the row
-    for (int u = wid; u < sh.ncand; u += NT / 32) {
-      const int pos = cand_pos[u];
-      const uint32_t key = cand_key[u];
-      const int gi = lo + pos;
-      int beat = 0;
-      for (int m = lane; m < incand; m += 32) {
-        const uint32_t km = sh.all_key[m];
-        beat += (km > key) || (km == key && sh.all_idx[m] < gi);
+    if (mode == 1) {
+      // ---- C1: gather all candidates of the cluster (all loads in flight)
+      int coff[CS + 1];
+      coff[0] = 0;
+#pragma unroll
+      for (int c = 0; c < CS; ++c) coff[c + 1] = coff[c] + sh.peer_nc[c];
+      for (int m = tid; m < coff[CS]; m += NT) {
+        int c = 0;
+#pragma unroll
+        for (int cc = 1; cc < CS; ++cc) c += m >= coff[cc];
+        const int u = m - coff[c];
+        sh.all_key[m] = peer_ptr<CS>(cand_key, c)[u];
+        sh.all_idx[m] = min(v, c * per) + peer_ptr<CS>(cand_pos, c)[u];
+        sh.all_cta[m] = (unsigned char)c;
       }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) beat += __shfl_xor_sync(0xffffffffu, beat, o);
-      if (lane == 0 && beat < need) atomicOr(&selbits[pos >> 5], 1u << (pos & 31));
-    }
-    __syncthreads();
-  } else if (mode == 2) {
-    // ---- C2: radix select among the keys of b* (degenerate distributions)
-    cluster_barrier<CS>();  // peers are done reading sh.hist
-    need_eq = need;
-    // the 12 leading bits are b*; digits of bits 19..12, 11..4, 3..0
-    pmask = 0xFFF00000u;
-    pval = (uint32_t)bstar << 20;
-    const int shift0 = 12, npass = 3;
-    for (int pass = 0; pass < npass; ++pass) {
-      const int shift = shift0 - 8 * pass;
-      const int sh_ = shift < 0 ? 0 : shift;
-      const uint32_t dmask = shift < 0 ? 15u : 255u;  // the last fixed-bin digit has 4 bits
-      int *h = sh.hist + 256 * (pass & 1);
-      for (int j = tid; j < 256; j += NT) h[j] = 0;
+      for (int j = tid; j < 256; j += NT) sh.hist[j] = 0;
       __syncthreads();
-      for (int j0 = 0; j0 < len; j0 += NT) {
-        const int j = j0 + tid;
-        const uint32_t key = j < len ? keys[j] : 0u;
-        const bool ok = j < len && (key & pmask) == pval;
-        const unsigned act = __ballot_sync(0xffffffffu, ok);
-        if (ok) {
-          const uint32_t dg = (key >> sh_) & dmask;
-          const unsigned same = __match_any_sync(act, dg);
-          if (lane == __ffs(same) - 1) atomicAdd(&h[dg], __popc(same));
+      // radix step on bits 19..12 of the candidates (all share bits 31..20)
+      for (int m = tid; m < incand; m += NT) atomicAdd(&sh.hist[(sh.all_key[m] >> 12) & 255u], 1);
+      __syncthreads();
+      find_bucket(sh, 256, need, tid < 256 ? sh.hist[255 - tid] : 0);
+      const uint32_t dstar = (uint32_t)sh.info[0];
+      const int need2 = need - sh.info[1];  // to take from sub-bin d*
+      const int nsub = sh.info[2];          // candidates in sub-bin d*
+      // the members of d* in a short list (sh.hist as scratch)
+      uint32_t *sub_key = reinterpret_cast<uint32_t *>(sh.hist);
+      int *sub_idx = sh.hist + kTopkRankCap;
+      if (tid == 0) sh.info[3] = 0;
+      __syncthreads();
+      for (int m = tid; m < incand; m += NT) {
+        if (((sh.all_key[m] >> 12) & 255u) == dstar) {
+          const int u = atomicAdd(&sh.info[3], 1);
+          sub_key[u] = sh.all_key[m];
+          sub_idx[u] = sh.all_idx[m];
         }
       }
-      cluster_barrier<CS>();
-      int c2 = 0;
-      if (tid < 256) {
-        const int dg = 255 - tid;
-#pragma unroll
-        for (int c = 0; c < CS; ++c) c2 += peer_ptr<CS>(&sh, c)->hist[256 * (pass & 1) + dg];
-      }
-      int tot2;
-      const int ab2 = block_exclusive_scan(c2, sh.scan, &tot2);
-      if (tid < 256 && ab2 < need_eq && ab2 + c2 >= need_eq) {
-        sh.info[0] = 255 - tid;
-        sh.info[1] = ab2;
-        sh.info[2] = c2;
+      __syncthreads();
+      // every candidate's fate: above d* in, below out, inside ranked
+      // pairwise; own ones into selbits, and per-CTA counts
+      for (int m = tid; m < incand; m += NT) {
+        const uint32_t key = sh.all_key[m];
+        const uint32_t d = (key >> 12) & 255u;
+        bool sel = d > dstar;
+        if (d == dstar) {
+          const int gi = sh.all_idx[m];
+          int beat = 0;
+          for (int q = 0; q < nsub; ++q) {
+            const uint32_t kq = sub_key[q];
+            beat += (kq > key) || (kq == key && sub_idx[q] < gi);
+          }
+          sel = beat < need2;
+        }
+        if (sel) {
+          const int c = sh.all_cta[m];
+          atomicAdd(&sh.peer_sel[c], 1);
+          if (c == rank) {
+            const int pos = sh.all_idx[m] - lo;
+            atomicOr(&selbits[pos >> 5], 1u << (pos & 31));
+          }
+        }
       }
       __syncthreads();
-      need_eq -= sh.info[1];
-      pmask |= dmask << sh_;
-      pval |= (uint32_t)sh.info[0] << sh_;
-      const bool done = (sh.info[2] == need_eq);
-      __syncthreads();  // info is read by every thread before the next pass rewrites it
-      if (done) {
-        all_eq = true;
-        break;
-      }
     }
+    // ---- D: offsets from the counts, then the indices from the bit masks
+    int off = 0;
+#pragma unroll
+    for (int c = 0; c < CS; ++c)
+      if (c < rank) off += sh.peer_above[c] + sh.peer_sel[c];
+    int n_sel = 0;  // this warp's selected keys
+    for (int g = w0 + 32 * lane; g < w1; g += 32 * 32) n_sel += __popc(abovebits[g >> 5] | selbits[g >> 5]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) n_sel += __shfl_xor_sync(0xffffffffu, n_sel, o);
+    int cta_sel;
+    const int before = block_exclusive_scan(lane == 0 ? n_sel : 0, sh.scan, &cta_sel);
+    int pos = off + __shfl_sync(0xffffffffu, before, 0);
+    for (int g = w0; g < w1; g += 32) {
+      const unsigned mall = abovebits[g >> 5] | selbits[g >> 5];
+      if ((mall >> lane) & 1u) {
+        const int p = pos + __popc(mall & lt);
+        // (p < k always holds: exactly k keys are selected; the guard keeps a
+        // miscount from ever writing outside the row)
+        if (p < k) orow[p] = lo + g + lane;
+      }
+      pos += __popc(mall);
+    }
+    cluster_barrier<CS>();  // [3] peers may still read this CTA's shared memory
+    return;
   }
 
-  // ---- D: count, exchange offsets, write in index order
-  // classify (mode 2): 1 selected, 2 tied at the radix threshold, 0 not
+  // ---- fallback (mode 2): cluster-wide radix select among the keys of b*,
+  // on bits 19..12, 11..4, 3..0, ties by index
+  cluster_barrier<CS>();  // peers are done reading sh.hist
+  int need_eq = need;
+  uint32_t pmask = 0xFFF00000u, pval = (uint32_t)bstar << 20;
+  bool all_eq = false;
+  for (int pass = 0; pass < 3; ++pass) {
+    const int shift = 12 - 8 * pass;
+    const int sh_ = shift < 0 ? 0 : shift;
+    const uint32_t dmask = shift < 0 ? 15u : 255u;  // the last digit has 4 bits
+    int *h = sh.hist + 256 * (pass & 1);
+    for (int j = tid; j < 256; j += NT) h[j] = 0;
+    __syncthreads();
+    for (int j0 = 0; j0 < len; j0 += NT) {
+      const int j = j0 + tid;
+      const uint32_t key = j < len ? keys[j] : 0u;
+      const bool ok = j < len && (key & pmask) == pval;
+      const unsigned act = __ballot_sync(0xffffffffu, ok);
+      if (ok) {
+        const uint32_t dg = (key >> sh_) & dmask;
+        const unsigned same = __match_any_sync(act, dg);
+        if (lane == __ffs(same) - 1) atomicAdd(&h[dg], __popc(same));
+      }
+    }
+    cluster_barrier<CS>();
+    int c2 = 0;
+    if (tid < 256) {
+#pragma unroll
+      for (int c = 0; c < CS; ++c) c2 += peer_ptr<CS>(&sh, c)->hist[256 * (pass & 1) + 255 - tid];
+    }
+    find_bucket(sh, 256, need_eq, c2);
+    need_eq -= sh.info[1];
+    pmask |= dmask << sh_;
+    pval |= (uint32_t)sh.info[0] << sh_;
+    const bool done = (sh.info[2] == need_eq);
+    __syncthreads();  // info is read by every thread before the next pass rewrites it
+    if (done) {
+      all_eq = true;
+      break;
+    }
+  }
+  // classify: 1 selected, 2 tied at the radix threshold, 0 not
   auto classify = [&](int j) -> int {
     const uint32_t key = keys[j];
     const int bn = score_bin(key);
@@ -360,15 +416,11 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(const float *__restrict__
     return 0;
   };
   int n_sel = 0, n_eq = 0;  // warp totals (identical in every lane)
-  if (mode != 2) {
-    for (int g = w0; g < w1; g += 32) n_sel += __popc(abovebits[g >> 5] | selbits[g >> 5]);
-  } else {
-    for (int g = w0; g < w1; g += 32) {
-      const int j = g + lane;
-      const int cl = j < w1 ? classify(j) : 0;
-      n_sel += __popc(__ballot_sync(0xffffffffu, cl == 1));
-      n_eq += __popc(__ballot_sync(0xffffffffu, cl == 2));
-    }
+  for (int g = w0; g < w1; g += 32) {
+    const int j = g + lane;
+    const int cl = j < w1 ? classify(j) : 0;
+    n_sel += __popc(__ballot_sync(0xffffffffu, cl == 1));
+    n_eq += __popc(__ballot_sync(0xffffffffu, cl == 2));
   }
   int cta_sel, cta_eq;
   const int sel_before = block_exclusive_scan(lane == 0 ? n_sel : 0, sh.scan, &cta_sel);
@@ -378,11 +430,16 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(const float *__restrict__
     sh.cta_counts[1] = cta_eq;
   }
   cluster_barrier<CS>();
+  if (tid < CS) {
+    const TopkShared *p = peer_ptr<CS>(&sh, tid);
+    sh.peer_above[tid] = p->cta_counts[0];
+    sh.peer_nc[tid] = p->cta_counts[1];
+  }
+  __syncthreads();
   int off = 0, eq_seen = 0, take_eq = 0;
 #pragma unroll
   for (int c = 0; c < CS; ++c) {
-    const TopkShared *p = peer_ptr<CS>(&sh, c);
-    const int g = p->cta_counts[0], e = p->cta_counts[1];
+    const int g = sh.peer_above[c], e = sh.peer_nc[c];
     const int te = max(0, min(e, need_eq - eq_seen));
     if (c < rank) off += g + te;
     if (c == rank) take_eq = te;
@@ -395,26 +452,19 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(const float *__restrict__
   int pos = off + wsel + max(0, min(weq, take_eq));
   int eq_rank = weq;
   for (int g = w0; g < w1; g += 32) {
-    unsigned mall;
-    if (mode != 2) {
-      mall = abovebits[g >> 5] | selbits[g >> 5];
-    } else {
-      const int j = g + lane;
-      const int cl = j < w1 ? classify(j) : 0;
-      const unsigned ms = __ballot_sync(0xffffffffu, cl == 1);
-      const unsigned me = __ballot_sync(0xffffffffu, cl == 2);
-      // tied keys are taken in index order while eq_rank < take_eq
-      const int te_here = max(0, min(__popc(me), take_eq - eq_rank));
-      unsigned mt = me;  // keep the first te_here tied keys of this group
-      for (int d = __popc(me) - te_here; d > 0; --d) mt &= ~(1u << (31 - __clz(mt)));
-      mall = ms | mt;
-      eq_rank += __popc(me);
-    }
+    const int j = g + lane;
+    const int cl = j < w1 ? classify(j) : 0;
+    const unsigned ms = __ballot_sync(0xffffffffu, cl == 1);
+    const unsigned me = __ballot_sync(0xffffffffu, cl == 2);
+    // tied keys are taken in index order while eq_rank < take_eq
+    const int te_here = max(0, min(__popc(me), take_eq - eq_rank));
+    unsigned mt = me;  // keep the first te_here tied keys of this group
+    for (int d = __popc(me) - te_here; d > 0; --d) mt &= ~(1u << (31 - __clz(mt)));
+    const unsigned mall = ms | mt;
+    eq_rank += __popc(me);
     if ((mall >> lane) & 1u) {
       const int p = pos + __popc(mall & lt);
-      // (p < k always holds: exactly k keys are selected; the guard keeps a
-      // miscount from ever writing outside the row)
-      if (p < k) orow[p] = lo + g + lane;
+      if (p < k) orow[p] = lo + j;
     }
     pos += __popc(mall);
   }
