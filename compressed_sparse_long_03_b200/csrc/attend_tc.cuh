@@ -21,8 +21,10 @@
 //           A = P, B = the SAME key tile read MN-major (the entry is the value);
 //   accumulate  O is read back per lane and folded into registers with the
 //           running rescale.
-// The CTAs' partial (max, sum, output) merge through distributed shared
-// memory in fixed rank order, as in the CUDA-core kernel.
+// Each CTA pushes its partial (max, sum, output) of every head into the
+// shared memory of the CTA that finalises that head (distributed shared
+// memory stores); after one cluster barrier each CTA merges its heads in
+// fixed rank order from local memory.
 #pragma once
 
 #include <cooperative_groups.h>
@@ -34,11 +36,13 @@
 namespace csa {
 
 constexpr int kAtThreads = 128;
-constexpr int kAtMaxTile = 256;                      // keys per tile
+constexpr int kAtMaxTile = 192;                      // keys per tile
 constexpr uint32_t kAtQAtom = 128 * 128;             // 128 rows x 128 B
 constexpr uint32_t kAtKHalf = kAtMaxTile * 128;      // one 64-wide d slice of the key tile
 constexpr uint32_t kAtPAtom = 128 * 128;             // 128 heads x 64 keys x 2 B
-constexpr size_t kAtSmem = 1024 + 2 * kAtQAtom + 2 * kAtKHalf + 4 * kAtPAtom;
+constexpr uint32_t kAtPart = 128 * 128 * 4;          // partial outputs pushed by the cluster
+constexpr size_t kAtSmem =
+    1024 + 2 * kAtQAtom + 2 * kAtKHalf + (kAtMaxTile / 64) * kAtPAtom + kAtPart;
 
 template <int CS>
 __global__ void __launch_bounds__(kAtThreads, 1) k_attend_tc(AttendArgs a) {
@@ -49,8 +53,8 @@ __global__ void __launch_bounds__(kAtThreads, 1) k_attend_tc(AttendArgs a) {
   __shared__ uint64_t bar_s, bar_o;
   __shared__ int kvalid[kAtMaxTile / 32];  // validity bits, one word per 32 keys
   __shared__ const __nv_bfloat16 *rowp[kAtMaxTile];
-  __shared__ float pm[128], pl[128];
-  __shared__ float mw[136], minv[128];  // merge weights [head][rank], 1 / sum
+  __shared__ float pm[136], pl[136];   // pushed partial max / sum [hl * CS + c]
+  __shared__ float mw[136], minv[128];  // merge weights [hl * CS + c], 1 / sum
   __shared__ int abort_flag;
 
   uint8_t *base = reinterpret_cast<uint8_t *>(
@@ -58,7 +62,9 @@ __global__ void __launch_bounds__(kAtThreads, 1) k_attend_tc(AttendArgs a) {
   uint8_t *sQ = base;
   uint8_t *sK = sQ + 2 * kAtQAtom;
   uint8_t *sP = sK + 2 * kAtKHalf;
-  float *part = reinterpret_cast<float *>(base);  // [128][128] partial outputs, after the loop
+  // partials of the heads this CTA finalises, written by every CTA of the
+  // cluster: [head slot hl][source rank c][128] (slot hl = head h / CS)
+  float *part = reinterpret_cast<float *>(sP + (kAtMaxTile / 64) * kAtPAtom);
 
   const int rank = (CS > 1) ? (int)cg::this_cluster().block_rank() : 0;
   const int r = blockIdx.x / CS;
@@ -257,31 +263,29 @@ __global__ void __launch_bounds__(kAtThreads, 1) k_attend_tc(AttendArgs a) {
     __syncthreads();  // every lane done with S, P and O before they are rewritten
   }
 
-  // ---- publish partials: row h of `part` holds head h's output as 32
-  // float4 slots rotated by h (conflict-free stores, float4 peer reads)
-  __syncthreads();
+  // ---- push this CTA's partial (max, sum, output) of head h into the CTA
+  // that finalises h (rank h % CS), one cluster barrier, merge locally
   if (tid < H) {
-    pm[tid] = m_run;
-    pl[tid] = l_run;
-    float4 *prow = reinterpret_cast<float4 *>(part + (size_t)tid * D);
+    const int own = tid % CS, slot = (tid / CS) * CS + rank;
+    float4 *dst = reinterpret_cast<float4 *>(att_peer<CS>(part, own) + (size_t)slot * D);
 #pragma unroll
-    for (int j = 0; j < D / 4; ++j)
-      prow[(j + tid) & (D / 4 - 1)] = make_float4(o[4 * j], o[4 * j + 1], o[4 * j + 2], o[4 * j + 3]);
+    for (int j = 0; j < D / 4; ++j) dst[j] = make_float4(o[4 * j], o[4 * j + 1], o[4 * j + 2], o[4 * j + 3]);
+    att_peer<CS>(pm, own)[slot] = m_run;
+    att_peer<CS>(pl, own)[slot] = l_run;
   }
   att_cluster_sync<CS>();
   // merge weights of this CTA's heads (h = rank + CS * hl), ranks in order
   const int nmine = (H - rank + CS - 1) / CS;
   if (tid < nmine) {
-    const int h = rank + CS * tid;
     float M = -INFINITY;
 #pragma unroll
-    for (int c = 0; c < CS; ++c) M = fmaxf(M, att_peer<CS>(pm, c)[h]);
+    for (int c = 0; c < CS; ++c) M = fmaxf(M, pm[tid * CS + c]);
     float Ls = 0.f;
 #pragma unroll
     for (int c = 0; c < CS; ++c) {
-      const float mc = att_peer<CS>(pm, c)[h];
+      const float mc = pm[tid * CS + c];
       const float wgt = (mc == -INFINITY) ? 0.f : ex2(mc - M);
-      Ls = fmaf(att_peer<CS>(pl, c)[h], wgt, Ls);
+      Ls = fmaf(pl[tid * CS + c], wgt, Ls);
       mw[tid * CS + c] = wgt;
     }
     minv[tid] = 1.f / Ls;
@@ -295,7 +299,7 @@ __global__ void __launch_bounds__(kAtThreads, 1) k_attend_tc(AttendArgs a) {
     for (int c = 0; c < CS; ++c) {
       const float wgt = mw[hl * CS + c];
       if (wgt == 0.f) continue;
-      const float4 p = reinterpret_cast<const float4 *>(att_peer<CS>(part, c) + (size_t)h * D)[(j + h) & (D / 4 - 1)];
+      const float4 p = reinterpret_cast<const float4 *>(part + (size_t)(hl * CS + c) * D)[j];
       acc.x = fmaf(p.x, wgt, acc.x);
       acc.y = fmaf(p.y, wgt, acc.y);
       acc.z = fmaf(p.z, wgt, acc.z);
@@ -309,7 +313,6 @@ __global__ void __launch_bounds__(kAtThreads, 1) k_attend_tc(AttendArgs a) {
     pk.y = *reinterpret_cast<uint32_t *>(&hi2);
     *reinterpret_cast<uint2 *>(out + (size_t)h * D + 4 * j) = pk;
   }
-  att_cluster_sync<CS>();
   if (tid == 0 && abort_flag) raise_dev_err(kDevErrTimeout);
   tc_fence_before();
   __syncthreads();

@@ -246,24 +246,36 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(const float *__restrict__
   if (mode != 2) {
     // ---- C: decided keys into abovebits, candidates into the list
     int my_above = 0;
-    for (int g = w0; g < w1; g += 32) {
-      const int j = g + lane;
-      const int bn = j < w1 ? score_bin(keys[j]) : -1;
-      const unsigned ma = __ballot_sync(0xffffffffu, mode == 0 ? bn >= bstar : bn > bstar);
-      const unsigned mc = __ballot_sync(0xffffffffu, mode == 1 && bn == bstar);
-      if (lane == 0) {
-        abovebits[g >> 5] = ma;
-        selbits[g >> 5] = 0u;
+    constexpr int GU = 4;  // groups per iteration: independent loads in flight
+    for (int g0 = w0; g0 < w1; g0 += 32 * GU) {
+      uint32_t kk[GU];
+#pragma unroll
+      for (int i = 0; i < GU; ++i) {
+        const int j = g0 + 32 * i + lane;
+        kk[i] = j < w1 ? keys[j] : 0u;
       }
-      my_above += __popc(ma);
-      if (mc) {
-        int base = 0;
-        if (lane == 0) base = atomicAdd(&sh.ncand, __popc(mc));
-        base = __shfl_sync(0xffffffffu, base, 0);
-        if ((mc >> lane) & 1u) {
-          const int u = base + __popc(mc & lt);
-          cand_key[u] = keys[j];
-          cand_pos[u] = j;
+#pragma unroll
+      for (int i = 0; i < GU; ++i) {
+        const int g = g0 + 32 * i;
+        if (g >= w1) break;  // warp-uniform
+        const int j = g + lane;
+        const int bn = j < w1 ? score_bin(kk[i]) : -1;
+        const unsigned ma = __ballot_sync(0xffffffffu, mode == 0 ? bn >= bstar : bn > bstar);
+        const unsigned mc = __ballot_sync(0xffffffffu, mode == 1 && bn == bstar);
+        if (lane == 0) {
+          abovebits[g >> 5] = ma;
+          selbits[g >> 5] = 0u;
+        }
+        my_above += __popc(ma);
+        if (mc) {
+          int base = 0;
+          if (lane == 0) base = atomicAdd(&sh.ncand, __popc(mc));
+          base = __shfl_sync(0xffffffffu, base, 0);
+          if ((mc >> lane) & 1u) {
+            const int u = base + __popc(mc & lt);
+            cand_key[u] = kk[i];
+            cand_pos[u] = j;
+          }
         }
       }
     }
@@ -350,15 +362,24 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(const float *__restrict__
     int cta_sel;
     const int before = block_exclusive_scan(lane == 0 ? n_sel : 0, sh.scan, &cta_sel);
     int pos = off + __shfl_sync(0xffffffffu, before, 0);
-    for (int g = w0; g < w1; g += 32) {
-      const unsigned mall = abovebits[g >> 5] | selbits[g >> 5];
-      if ((mall >> lane) & 1u) {
-        const int p = pos + __popc(mall & lt);
-        // (p < k always holds: exactly k keys are selected; the guard keeps a
-        // miscount from ever writing outside the row)
-        if (p < k) orow[p] = lo + g + lane;
+    for (int g0 = w0; g0 < w1; g0 += 32 * 4) {
+      unsigned mw[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int g = g0 + 32 * i;
+        mw[i] = g < w1 ? (abovebits[g >> 5] | selbits[g >> 5]) : 0u;
       }
-      pos += __popc(mall);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const unsigned mall = mw[i];
+        if ((mall >> lane) & 1u) {
+          const int p = pos + __popc(mall & lt);
+          // (p < k always holds: exactly k keys are selected; the guard keeps
+          // a miscount from ever writing outside the row)
+          if (p < k) orow[p] = lo + g0 + 32 * i + lane;
+        }
+        pos += __popc(mall);
+      }
     }
     cluster_barrier<CS>();  // [3] peers may still read this CTA's shared memory
     return;
