@@ -63,11 +63,12 @@ struct TopkShared {
 };
 
 // Dynamic shared memory of one CTA for slices of up to `per` keys: the keys
-// (plus alignment slack), the candidates (key and position) and two bit
-// masks over the slice (keys above the threshold bin, chosen candidates).
+// (plus alignment slack), the candidates (key and position), two bit masks
+// over the slice (keys above the threshold bin, chosen candidates) and the
+// largest bin of every 32-key group.
 __host__ __device__ constexpr size_t topk_dyn_bytes(int per) {
   return 4ull * ((size_t)per + 4 + 2 * (size_t)(per < kTopkRankCap ? per : kTopkRankCap) +
-                 2 * (((size_t)per + 31) / 32));
+                 3 * (((size_t)per + 3 + 31) / 32));
 }
 
 template <int CS>
@@ -140,16 +141,21 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(const float *__restrict__
   const int lo = min(v, rank * per), hi = min(v, lo + per);
   const int len = hi - lo;
   const int ccap = per < kTopkRankCap ? per : kTopkRankCap;
-  const int nwords = (per + 31) / 32;
   const float *srow = scores + (size_t)r * nc_max;
   // the slice start's misalignment to 16 B, mirrored in the key array so that
-  // vector loads and vector stores line up
+  // vector loads and vector stores line up.  Key j sits at position
+  // P = j + p0 of the array; groups of 32 positions (one bit-mask word each)
+  // never split a 16-byte vector.
   const int head0 = (int)((16 - (reinterpret_cast<uintptr_t>(srow + lo) & 15)) & 15) / 4;
-  uint32_t *keys = dyn + ((4 - head0) & 3);                       // [per], keys+head0 16 B aligned
+  const int p0 = (4 - head0) & 3;
+  const int nwords = (per + 3 + 31) / 32;
+  const int ngroups = (p0 + len + 31) / 32;
+  uint32_t *keys = dyn + p0;                                      // [per], keys+head0 16 B aligned
   uint32_t *cand_key = dyn + per + 4;                             // [ccap]
   int *cand_pos = reinterpret_cast<int *>(dyn + per + 4 + ccap);  // [ccap]
   uint32_t *selbits = dyn + per + 4 + 2 * ccap;                   // [nwords] chosen candidates
   uint32_t *abovebits = selbits + nwords;                         // [nwords] decided above b*
+  uint32_t *gmaxbin = abovebits + nwords;                         // [nwords] largest bin of a group
 
   for (int j = tid; j < kScoreBins; j += NT) sh.hist[j] = 0;
   if (tid < kTopkSuper) sh.super[tid] = 0;
@@ -158,6 +164,7 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(const float *__restrict__
     sh.above = 0;
   }
   if (tid < 16) sh.peer_sel[tid] = 0;
+  for (int j = tid; j < 3 * nwords; j += NT) selbits[j] = 0u;  // both masks and group maxima
   __syncthreads();
 
   // ---- A: keys (16-byte vector loads, eight in flight per thread) and the
@@ -169,6 +176,7 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(const float *__restrict__
       const uint32_t key = order_key(f);
       keys[j] = key;
       atomicAdd(&sh.hist[score_bin(key)], 1);
+      atomicMax(&gmaxbin[(j + p0) >> 5], (uint32_t)score_bin(key));
     };
     for (int j = tid; j < head; j += NT) take(j, __ldg(src + j));
     const int nvec = (len - head) / 4;
@@ -189,10 +197,13 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(const float *__restrict__
           const uint4 kv = make_uint4(order_key(f[i].x), order_key(f[i].y), order_key(f[i].z),
                                       order_key(f[i].w));
           vkeys[u] = kv;
-          atomicAdd(&sh.hist[score_bin(kv.x)], 1);
-          atomicAdd(&sh.hist[score_bin(kv.y)], 1);
-          atomicAdd(&sh.hist[score_bin(kv.z)], 1);
-          atomicAdd(&sh.hist[score_bin(kv.w)], 1);
+          const int b0 = score_bin(kv.x), b1 = score_bin(kv.y), b2 = score_bin(kv.z),
+                    b3 = score_bin(kv.w);
+          atomicAdd(&sh.hist[b0], 1);
+          atomicAdd(&sh.hist[b1], 1);
+          atomicAdd(&sh.hist[b2], 1);
+          atomicAdd(&sh.hist[b3], 1);
+          atomicMax(&gmaxbin[(head + 4 * u + p0) >> 5], (uint32_t)max(max(b0, b1), max(b2, b3)));
         }
       }
     }
@@ -238,44 +249,32 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(const float *__restrict__
   // candidates; 2 the cluster-wide radix fallback
   const int mode = (incand == need) ? 0 : (incand <= kTopkRankCap ? 1 : 2);
 
-  // warp w owns the contiguous chunk [w*cw, (w+1)*cw) of the slice, walked in
-  // groups of 32 consecutive keys (group g = bit-mask word g/32)
-  const int cw = ((len + NW - 1) / NW + 31) & ~31;
-  const int w0 = min(len, wid * cw), w1 = min(len, w0 + cw);
+  // warp w owns a contiguous run of 32-position groups [G0, G1); a group
+  // whose largest bin is below b* holds nothing to select and is skipped
+  const int gpw = (ngroups + NW - 1) / NW;
+  const int G0 = min(ngroups, wid * gpw), G1 = min(ngroups, G0 + gpw);
 
   if (mode != 2) {
     // ---- C: decided keys into abovebits, candidates into the list
     int my_above = 0;
-    constexpr int GU = 4;  // groups per iteration: independent loads in flight
-    for (int g0 = w0; g0 < w1; g0 += 32 * GU) {
-      uint32_t kk[GU];
-#pragma unroll
-      for (int i = 0; i < GU; ++i) {
-        const int j = g0 + 32 * i + lane;
-        kk[i] = j < w1 ? keys[j] : 0u;
-      }
-#pragma unroll
-      for (int i = 0; i < GU; ++i) {
-        const int g = g0 + 32 * i;
-        if (g >= w1) break;  // warp-uniform
-        const int j = g + lane;
-        const int bn = j < w1 ? score_bin(kk[i]) : -1;
-        const unsigned ma = __ballot_sync(0xffffffffu, mode == 0 ? bn >= bstar : bn > bstar);
-        const unsigned mc = __ballot_sync(0xffffffffu, mode == 1 && bn == bstar);
-        if (lane == 0) {
-          abovebits[g >> 5] = ma;
-          selbits[g >> 5] = 0u;
-        }
-        my_above += __popc(ma);
-        if (mc) {
-          int base = 0;
-          if (lane == 0) base = atomicAdd(&sh.ncand, __popc(mc));
-          base = __shfl_sync(0xffffffffu, base, 0);
-          if ((mc >> lane) & 1u) {
-            const int u = base + __popc(mc & lt);
-            cand_key[u] = kk[i];
-            cand_pos[u] = j;
-          }
+    for (int G = G0; G < G1; ++G) {
+      if ((int)gmaxbin[G] < bstar) continue;  // warp-uniform
+      const int j = 32 * G + lane - p0;
+      const bool in = j >= 0 && j < len;
+      const uint32_t key = in ? keys[j] : 0u;
+      const int bn = in ? score_bin(key) : -1;
+      const unsigned ma = __ballot_sync(0xffffffffu, mode == 0 ? bn >= bstar : bn > bstar);
+      const unsigned mc = __ballot_sync(0xffffffffu, mode == 1 && bn == bstar);
+      if (lane == 0) abovebits[G] = ma;
+      my_above += __popc(ma);
+      if (mc) {
+        int base = 0;
+        if (lane == 0) base = atomicAdd(&sh.ncand, __popc(mc));
+        base = __shfl_sync(0xffffffffu, base, 0);
+        if ((mc >> lane) & 1u) {
+          const int u = base + __popc(mc & lt);
+          cand_key[u] = key;
+          cand_pos[u] = j;
         }
       }
     }
@@ -343,8 +342,8 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(const float *__restrict__
           const int c = sh.all_cta[m];
           atomicAdd(&sh.peer_sel[c], 1);
           if (c == rank) {
-            const int pos = sh.all_idx[m] - lo;
-            atomicOr(&selbits[pos >> 5], 1u << (pos & 31));
+            const int P = sh.all_idx[m] - lo + p0;
+            atomicOr(&selbits[P >> 5], 1u << (P & 31));
           }
         }
       }
@@ -356,35 +355,30 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(const float *__restrict__
     for (int c = 0; c < CS; ++c)
       if (c < rank) off += sh.peer_above[c] + sh.peer_sel[c];
     int n_sel = 0;  // this warp's selected keys
-    for (int g = w0 + 32 * lane; g < w1; g += 32 * 32) n_sel += __popc(abovebits[g >> 5] | selbits[g >> 5]);
+    for (int G = G0 + lane; G < G1; G += 32) n_sel += __popc(abovebits[G] | selbits[G]);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) n_sel += __shfl_xor_sync(0xffffffffu, n_sel, o);
     int cta_sel;
     const int before = block_exclusive_scan(lane == 0 ? n_sel : 0, sh.scan, &cta_sel);
     int pos = off + __shfl_sync(0xffffffffu, before, 0);
-    for (int g0 = w0; g0 < w1; g0 += 32 * 4) {
-      unsigned mw[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int g = g0 + 32 * i;
-        mw[i] = g < w1 ? (abovebits[g >> 5] | selbits[g >> 5]) : 0u;
+    for (int G = G0; G < G1; ++G) {
+      const unsigned mall = abovebits[G] | selbits[G];
+      if (mall == 0u) continue;  // warp-uniform
+      if ((mall >> lane) & 1u) {
+        const int p = pos + __popc(mall & lt);
+        // (p < k always holds: exactly k keys are selected; the guard keeps a
+        // miscount from ever writing outside the row)
+        if (p < k) orow[p] = lo + 32 * G + lane - p0;
       }
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const unsigned mall = mw[i];
-        if ((mall >> lane) & 1u) {
-          const int p = pos + __popc(mall & lt);
-          // (p < k always holds: exactly k keys are selected; the guard keeps
-          // a miscount from ever writing outside the row)
-          if (p < k) orow[p] = lo + g0 + 32 * i + lane;
-        }
-        pos += __popc(mall);
-      }
+      pos += __popc(mall);
     }
     cluster_barrier<CS>();  // [3] peers may still read this CTA's shared memory
     return;
   }
 
+  // key-index chunks of 32 keys per warp for the fallback's passes
+  const int cw = ((len + NW - 1) / NW + 31) & ~31;
+  const int w0 = min(len, wid * cw), w1 = min(len, w0 + cw);
   // ---- fallback (mode 2): cluster-wide radix select among the keys of b*,
   // on bits 19..12, 11..4, 3..0, ties by index
   cluster_barrier<CS>();  // peers are done reading sh.hist
