@@ -10,6 +10,7 @@ Entry points (method definitions are stated in ``include/csa.h``):
   csa_compress    CSA overlapping compressor (stride 4, 8-token windows)
   hca_compress    HCA compressor (stride m, no overlap)
   csa_index_topk  lightning-indexer scores + per-query top-k
+  csa_index_topk_noalloc  the same without a workspace (fixed device scratch)
   csa_attend      MQA attention over the selected entries + sliding window
   hca_attend      MQA attention over every visible HCA entry + sliding window
 """
@@ -58,12 +59,15 @@ def lib() -> ctypes.CDLL:
         L.csa_index_topk_workspace_size.argtypes = [I, I, I, I]
         L.csa_index_topk_workspace_size.restype = S
         L.csa_index_topk.argtypes = [P, P, P, P, P, I, I, I, I, I, I, I, P, P, P, S, P]
+        L.csa_index_topk_noalloc.argtypes = [P, P, P, P, P, I, I, I, I, I, I, I, P, P]
+        L.csa_index_topk_noalloc_max_elems.argtypes = []
+        L.csa_index_topk_noalloc_max_elems.restype = S
         L.csa_index_scores.argtypes = [P, P, P, P, P, I, I, I, I, I, I, P, P]
         L.csa_topk.argtypes = [P, P, P, I, I, I, I, P, P]
         L.csa_attend.argtypes = [P, P, P, I, P, P, P, I, I, I, I, I, I, I, F, I, P, P]
         L.hca_attend.argtypes = [P, P, P, I, P, P, I, I, I, I, I, I, I, F, I, P, P]
         for name in ("csa_check_device_error", "csa_compress", "hca_compress", "csa_index_topk",
-                     "csa_index_scores", "csa_topk", "csa_attend", "hca_attend"):
+                     "csa_index_topk_noalloc", "csa_index_scores", "csa_topk", "csa_attend", "hca_attend"):
             getattr(L, name).restype = I
         _lib = L
     return _lib
@@ -178,6 +182,27 @@ def csa_index_topk(q_idx, w, k_idx, lens, k, q_pos=None, idx_out=None, scores_ou
     _check(lib().csa_index_topk(_p(q_idx), _p(w), _p(k_idx), _i32(lens), _i32(q_pos), B, Tq, HI, dI,
                                 nc_max, k, _dt(q_idx), _i32(idx_out), _p(scores_out), _p(workspace),
                                 ws_bytes, _s(stream)))
+    return idx_out
+
+
+def index_topk_noalloc_max_elems() -> int:
+    """Largest B*Tq*nc_max that csa_index_topk_noalloc accepts."""
+    return int(lib().csa_index_topk_noalloc_max_elems())
+
+
+def csa_index_topk_noalloc(q_idx, w, k_idx, lens, k, idx_out, q_pos=None, stream=None):
+    """csa_index_topk for callers that may not allocate device memory: the
+    scores go to the library's fixed device scratch instead of a workspace,
+    and the caller passes idx_out [B][Tq][k] int32.  Neither this function
+    nor the C call allocates.  Calls share the scratch, so calls that overlap
+    on the GPU race; the first call on a device belongs before any stream
+    capture."""
+    B, Tq, HI, dI = q_idx.shape
+    nc_max = k_idx.shape[1]
+    if tuple(idx_out.shape) != (B, Tq, k) or idx_out.dtype != torch.int32:
+        raise ValueError("idx_out must be an int32 tensor of shape [B][Tq][k]")
+    _check(lib().csa_index_topk_noalloc(_p(q_idx), _p(w), _p(k_idx), _i32(lens), _i32(q_pos), B, Tq,
+                                        HI, dI, nc_max, k, _dt(q_idx), _i32(idx_out), _s(stream)))
     return idx_out
 
 

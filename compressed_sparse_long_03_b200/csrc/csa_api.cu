@@ -689,3 +689,94 @@ int hca_attend(const void *q, const void *kv_c, const void *kv_tok, int n_tok,
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// csa_index_topk_noalloc: csa_index_topk with its score scratch in a fixed
+// array of device memory that the library itself holds.
+//
+// For callers that may not allocate device memory while they run: a serving
+// engine that has handed nearly all of the GPU's memory to its own pool, a
+// custom allocator that forbids allocations outside it, or code running
+// where cudaMalloc / cudaFree would synchronise the device or are not
+// allowed.  It calls no cudaMalloc, cudaFree or other allocating routine.
+//
+// The array below is loaded with the library and every GPU that loads it
+// keeps it (8 MiB) until the process exits.  Host code must not hand its name
+// to a kernel (on the host that name stands for a host-side shadow, not for
+// the device memory): the device address comes from cudaGetSymbolAddress,
+// looked up once per device with that device current, on the first call
+// made on that device.  That lookup may load the module, so the first call
+// on a device should come before any stream capture.
+//
+// All calls share the one array and it keeps what the previous call left in
+// it.  Nothing in it needs to start at zero: the scoring kernel rewrites
+// every visible entry of every row before the selection reads it, and the
+// selection reads visible entries only.  Calls that overlap on the GPU (two
+// streams, two host threads) race on the array; the caller serialises them.
+// ---------------------------------------------------------------------------
+namespace {
+
+constexpr size_t kNoAllocScoreFloats = size_t(2) << 20;  // 8 MiB: B*Tq*nc_max <= 2,097,152
+
+static __device__ __align__(256) float g_noalloc_scores[kNoAllocScoreFloats];
+
+constexpr int kNoAllocMaxDevices = 64;
+std::mutex g_noalloc_mu;
+float *g_noalloc_ptr[kNoAllocMaxDevices] = {};
+
+// Device address of g_noalloc_scores on the current device (looked up once).
+int noalloc_scores_ptr(float **out, const char *what) {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail(CSA_ERR_CUDA, "%s: cudaGetDevice: %s", what, cudaGetErrorString(e));
+  if (dev < 0 || dev >= kNoAllocMaxDevices)
+    return fail(CSA_ERR_UNSUPPORTED, "%s: device ordinal %d >= %d", what, dev, kNoAllocMaxDevices);
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void *p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scores);
+    if (e != cudaSuccess || !p)
+      return fail(CSA_ERR_CUDA, "%s: cudaGetSymbolAddress on device %d: %s", what, dev,
+                  cudaGetErrorString(e));
+    g_noalloc_ptr[dev] = static_cast<float *>(p);
+  }
+  *out = g_noalloc_ptr[dev];
+  return CSA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t csa_index_topk_noalloc_max_elems(void) { return kNoAllocScoreFloats; }
+
+int csa_index_topk_noalloc(const void *q_idx, const void *w, const void *k_idx, const int32_t *lens,
+                           const int32_t *q_pos, int B, int Tq, int HI, int dI, int nc_max, int k,
+                           csa_dtype dt, int32_t *idx_out, void *stream) {
+  const char *what = "csa_index_topk_noalloc";
+  begin_call();
+  int rc = check_index_args(what, dt, B, Tq, HI, dI, nc_max);
+  if (rc) return rc;
+  rc = check_topk_args(what, B, Tq, nc_max, k);
+  if (rc) return rc;
+  if ((long)B * Tq == 0) return CSA_OK;
+  const size_t elems = (size_t)B * Tq * nc_max;
+  if (elems > kNoAllocScoreFloats)
+    return fail(CSA_ERR_WORKSPACE,
+                "%s: B*Tq*nc_max = %zu scores exceed the fixed scratch of %zu (8 MiB); "
+                "use csa_index_topk with a workspace",
+                what, elems, kNoAllocScoreFloats);
+  if (!q_idx || !w || !lens || !idx_out || (nc_max > 0 && !k_idx))
+    return fail(CSA_ERR_NULL, "%s: a required pointer is NULL", what);
+  if (!aligned16(q_idx) || !aligned16(w) || (k_idx && !aligned16(k_idx)))
+    return fail(CSA_ERR_ALIGN, "%s: tensors must be 16-byte aligned", what);
+  float *scores = nullptr;
+  rc = noalloc_scores_ptr(&scores, what);
+  if (rc) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  rc = index_scores_impl(q_idx, w, k_idx, lens, q_pos, B, Tq, HI, dI, nc_max, dt, scores, false, st);
+  if (rc) return rc;
+  return topk_impl(scores, lens, q_pos, B, Tq, nc_max, k, idx_out, st);
+}
+
+}  // extern "C"

@@ -187,6 +187,35 @@ CSA_API int csa_topk(const float *scores, const int32_t *lens, const int32_t *q_
                      int nc_max, int k, int32_t *idx_out, void *stream);
 
 /* ------------------------------------------------------------------------
+ * csa_index_topk_noalloc -- csa_index_topk without a caller workspace.
+ *
+ * The paper has no counterpart: this is a library convenience.  It serves
+ * callers that may not allocate device memory during a call (a serving
+ * engine whose memory pool already holds nearly all of the GPU, a custom
+ * allocator that forbids allocations outside its pool, code where
+ * cudaMalloc / cudaFree would synchronise the device).  It allocates
+ * nothing: the scores live in a fixed 8 MiB array of device memory that the
+ * library holds on every GPU that loads it, until the process exits.
+ *
+ * Arguments, supported sets, selection rule and idx_out as for
+ * csa_index_topk with scores_out NULL.  In addition:
+ *   - B * Tq * nc_max must not exceed csa_index_topk_noalloc_max_elems()
+ *     (2,097,152, e.g. 8 decode queries at 1M tokens); larger calls fail
+ *     with CSA_ERR_WORKSPACE and leave idx_out untouched.
+ *   - The first call on a device looks up the array's device address (it
+ *     may load the library's GPU code): make it before any stream capture.
+ *   - Every call shares the array: calls that overlap on the GPU (other
+ *     streams, other host threads) race and must be serialised by the
+ *     caller.  Nothing left in it by an earlier call affects a result.
+ * ---------------------------------------------------------------------- */
+CSA_API size_t csa_index_topk_noalloc_max_elems(void);
+
+CSA_API int csa_index_topk_noalloc(const void *q_idx, const void *w, const void *k_idx,
+                                   const int32_t *lens, const int32_t *q_pos, int B, int Tq,
+                                   int HI, int dI, int nc_max, int k, csa_dtype dt,
+                                   int32_t *idx_out, void *stream);
+
+/* ------------------------------------------------------------------------
  * csa_attend -- sparse MQA attention over the selected entries + window.
  *
  * Anatomy page, "The skeleton": one key-value head is shared by every query
