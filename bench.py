@@ -46,6 +46,9 @@ def parse():
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-steps", type=int, default=1, help="oracle steps for cpu_baseline")
+    p.add_argument("--workload", type=int, default=4, choices=[1, 2, 3, 4, 5],
+                   help="4 (default): the 1M CSA decode step; 1, 2, 3, 5: the other "
+                        "workloads, one measurement line each (single GPU)")
     return p.parse_args()
 
 
@@ -185,6 +188,16 @@ def run_ours(args, rank, world, dev):
     s = dict(wl.sizes)
     B, nc, k, window = s["B"], s["nc"], s["k"], s["window"]
     D = {n: to_dev(wl[n], f"cuda:{dev}") for n in ("kI", "kv", "win", "q", "qI", "w", "lens")}
+    # the step's query-side inputs live in one device buffer (views), so that
+    # the end-to-end pass moves them with a single host-to-device copy
+    qnames = ("q", "qI", "w")
+    pack = torch.empty(sum(D[n].numel() for n in qnames), dtype=torch.bfloat16, device=dev)
+    off = 0
+    for n in qnames:
+        sz = D[n].numel()
+        pack[off:off + sz].copy_(D[n].reshape(-1))
+        D[n] = pack[off:off + sz].view(D[n].shape)
+        off += sz
     idx = torch.empty(B, 1, k, dtype=torch.int32, device=dev)
     out = torch.empty(B, 1, s["H"], s["d"], dtype=torch.bfloat16, device=dev)
     ws = csa.index_topk_workspace(B, 1, nc, False, device=dev)  # the scores
@@ -236,20 +249,19 @@ def run_ours(args, rank, world, dev):
     csa.check_device_error()
     ms = t0.elapsed_time(t1) / K
 
-    # end to end through the public API from pinned host buffers: H2D of the
-    # step's query inputs, the three calls, D2H of the output
-    host = {n: torch.from_numpy(np.ascontiguousarray(wl[n]).view(np.int16)).pin_memory()
-            for n in ("q", "qI", "w")}
+    # end to end through the public API from pinned host buffers: one H2D
+    # copy of the step's query inputs (q, q_I, w packed), the two calls, one
+    # D2H copy of the output
+    host = torch.from_numpy(np.concatenate([np.ascontiguousarray(wl[n]).reshape(-1).view(np.int16)
+                                            for n in qnames])).pin_memory()
     out_h = torch.empty(out.shape, dtype=torch.bfloat16).pin_memory()
-    qd = {n: D[n] for n in ("q", "qI", "w")}
 
     def step_e2e():
-        for n in ("q", "qI", "w"):
-            qd[n].view(torch.int16).copy_(host[n], non_blocking=True)
+        pack.view(torch.int16).copy_(host, non_blocking=True)
         step()
         out_h.copy_(out, non_blocking=True)
 
-    h2d = sum(host[n].numel() * 2 for n in host)
+    h2d = host.numel() * 2
     d2h = out_h.numel() * 2
     for _ in range(3):
         step_e2e()
@@ -269,6 +281,172 @@ def run_ours(args, rank, world, dev):
     return dict(ms=ms, ms_e2e=ms_e2e, stage=stage, clocks=clocks, s=s, B=B, h2d=h2d, d2h=d2h,
                 launches=launches_per_step * K, wl=wl,
                 ms_staged=sum(statistics.mean(v) for v in stage.values()))
+
+
+# --------------------------------------------------------------------------
+# the other workloads: one device-timed line each
+# --------------------------------------------------------------------------
+def other_workload_plan(wid, wl, csa, torch, D):
+    """(step stages, unit, units per step, algorithmic bytes, flops, what a
+    step is) of workload `wid`; every array already on the device in D."""
+    s = wl.sizes
+    k, window = s.get("k"), s["window"]
+    e = 4 if wl.dt == "f32" else 2
+    if wid in (1, 2):
+        B, n, d, dI, H, HI, Tq = s["B"], s["n"], s["d"], s["dI"], s["H"], s["HI"], s["Tq"]
+        nc = s["nc"]
+        C = torch.empty(B, nc, d, dtype=D["x"].dtype, device="cuda")
+        KI = torch.empty(B, nc, dI, dtype=D["x"].dtype, device="cuda")
+        idx = torch.empty(B, Tq, k, dtype=torch.int32, device="cuda")
+        out = torch.empty(B, Tq, H, d, dtype=D["x"].dtype, device="cuda")
+        ws = csa.index_topk_workspace(B, Tq, nc, False)
+        stages = [
+            ("csa_compress (KV)", lambda: csa.csa_compress(D["x"], D["lens"], D["Wa"], D["Wb"], D["beta"], out=C)),
+            ("csa_compress (indexer keys)",
+             lambda: csa.csa_compress(D["kx"], D["lens"], D["kWa"], D["kWb"], D["kbeta"], out=KI)),
+            ("csa_index_topk", lambda: csa.csa_index_topk(D["qI"], D["w"], KI, D["lens"], k, idx_out=idx,
+                                                          workspace=ws)),
+            ("csa_attend", lambda: csa.csa_attend(D["q"], C, D["x"], idx, D["lens"], window=window, out=out)),
+        ]
+        t = np.arange(n - Tq, n)
+        vis = (t + 1) // 4
+        sel = np.minimum(vis, k)
+        win = np.minimum(window, t + 1)
+        flops = (2.0 * 2 * n * d * 2 * d + 2.0 * 2 * n * dI * 2 * dI      # compressors (logits, both series)
+                 + 2.0 * float(vis.sum()) * HI * dI                       # indexer
+                 + 4.0 * float((sel + win).sum()) * H * d)                # QK^T and PV
+        byts = e * (B * n * (d + dI) + B * nc * (d + dI)                  # tokens read, caches written
+                    + float(vis.sum()) * dI                               # indexer keys per query
+                    + float((sel + win).sum()) * d                        # gathered rows
+                    + Tq * (2 * H * d + HI * dI + HI))                    # q, q_I, w, out
+        unit = "tokens/s" if wid == 2 else "queries/s"
+        what = ("one prefill pass of the 8192-token sequence: both compressors, indexer + top-k "
+                "and attention for every token" if wid == 2 else
+                "one decode step with the caches rebuilt from the 1024 tokens: both compressors, "
+                "indexer + top-k, attention")
+        return stages, unit, B * Tq, byts, flops, what
+    if wid == 3:
+        B, H, d, m = s["B"], s["H"], s["d"], s["m"]
+        out = torch.empty(B, 1, H, d, dtype=torch.bfloat16, device="cuda")
+        stages = [("hca_attend", lambda: csa.hca_attend(D["q"], D["hkv"], D["win"], D["lens"], m=m,
+                                                        window=window, out=out))]
+        v = s["n"] // m
+        byts = B * ((v + window) * d * 2 + 2 * H * d * 2)
+        flops = 4.0 * B * (v + window) * H * d
+        return stages, "queries/s", B, byts, flops, "one HCA decode step of the 32 sequences"
+    if wid == 5:
+        B, H, d, dI, HI, m = s["B"], s["H"], s["d"], s["dI"], s["HI"], s["m"]
+        nc = s["nc"]
+        idx = torch.empty(B, 1, k, dtype=torch.int32, device="cuda")
+        out_c = torch.empty(B, 1, H, d, dtype=torch.bfloat16, device="cuda")
+        out_h = torch.empty(B, 1, H, d, dtype=torch.bfloat16, device="cuda")
+        ws = csa.index_topk_workspace(B, 1, nc, False)
+        stages = [
+            ("csa_index_topk", lambda: csa.csa_index_topk(D["qI"], D["w"], D["kI"], D["lens"], k,
+                                                          idx_out=idx, workspace=ws)),
+            ("csa_attend", lambda: csa.csa_attend(D["q"], D["kv"], D["win"], idx, D["lens"],
+                                                  window=window, out=out_c)),
+            ("hca_attend", lambda: csa.hca_attend(D["q2"], D["hkv"], D["win"], D["lens"], m=m,
+                                                  window=window, out=out_h)),
+        ]
+        lens = wl["lens"].astype(np.int64)
+        vis, hv = lens // 4, lens // m
+        sel = np.minimum(vis, k)
+        byts = 2 * float((vis * dI + (sel + window) * d + (hv + window) * d).sum()
+                         + B * (4 * H * d + HI * dI + HI))
+        flops = float((2.0 * vis * HI * dI + 4.0 * (sel + window) * H * d + 4.0 * (hv + window) * H * d).sum())
+        return stages, "queries/s", B, byts, flops, "one decode step of the CSA + HCA layer pair"
+    raise KeyError(wid)
+
+
+def run_other_workload(args):
+    """Device time of one step of workload 1, 2, 3 or 5 (inputs resident in
+    HBM; the L2 is flushed by a 256 MiB write before every timed step, and
+    CUDA events bracket the step alone)."""
+    import torch
+    import compressed_sparse_long_03_b200 as csa
+    from tests.helpers import to_dev
+    torch.cuda.set_device(0)
+    wid = args.workload
+    wl = W.make(wid)
+    D = {n: to_dev(wl[n]) for n in wl.arrays if n != "needle_pos"}
+    stages, unit, units, byts, flops, what = other_workload_plan(wid, wl, csa, torch, D)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+
+    def step():
+        for _, fn in stages:
+            fn()
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    csa.check_device_error()
+    K = args.steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    sampler = ClockSampler(smi_index(str(torch.cuda.get_device_properties(0).uuid), 0))
+    sampler.start()
+    for i in range(K):
+        flush.zero_()
+        ev[i][0].record()
+        step()
+        ev[i][1].record()
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    ms = statistics.median(a.elapsed_time(b) for a, b in ev)
+    per = {name: [] for name, _ in stages}
+    csa.set_kernel_timing(True)
+    for i in range(K):
+        flush.zero_()
+        for name, fn in stages:
+            fn()
+            per[name].append(sum(csa.kernel_timing()))
+    csa.set_kernel_timing(False)
+    torch.cuda.synchronize()
+    csa.check_device_error()
+    peaks = load_peaks()
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    tfl = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    gbs = byts / (ms * 1e-3) / 1e9
+    tfs = flops / (ms * 1e-3) / 1e12
+    line = {"metric": f"{wl.name}: {unit}", "value": units * 1000.0 / ms, "unit": unit, "n_gpus": 1,
+            "steps": K, "warmup": max(3, args.warmup), "ms_per_step": ms, "higher_is_better": True,
+            "dtype": wl.dt, "data": "synthetic (seeded PCG64)",
+            "config": {"workload": wl.name, "step": what,
+                       "l2": "flushed before every timed step (256 MiB write); events bracket the step"},
+            "algorithmic": {"bytes_per_step": byts, "flops_per_step": flops, "achieved_gbs": gbs,
+                            "frac_of_measured_hbm": gbs / hbm, "achieved_tflops": tfs,
+                            "frac_of_measured_bf16": tfs / tfl, "peak_source": peaks["source"]},
+            "stages_us": {k2: 1000 * statistics.median(v) for k2, v in per.items()},
+            "stages_note": "per-call medians with the library's kernel timing on (serialised)",
+            "clocks": clocks}
+    if wid == 3:
+        line["hca_compress"] = time_hca_compress(wl, csa, torch, flush, min(K, 20), hbm)
+    print(json.dumps(line))
+    return 0
+
+
+def time_hca_compress(wl, csa, torch, flush, K, hbm):
+    """The HCA compressor over the workload's 131,072 tokens per sequence
+    (all 32 sequences), timed like the step."""
+    from tests.helpers import to_dev
+    s = wl.sizes
+    tk = W.hca_tokens(wl.sizes["seed"], s["B"], s["n"], s["d"], wl.dt, m=s["m"])
+    x, Wm, beta, lens = (to_dev(tk[n]) for n in ("x", "W", "beta", "lens"))
+    out = torch.empty(s["B"], tk.sizes["nc"], s["d"], dtype=torch.bfloat16, device="cuda")
+    for _ in range(3):
+        csa.hca_compress(x, lens, Wm, beta, m=s["m"], out=out)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    for i in range(K):
+        flush.zero_()
+        ev[i][0].record()
+        csa.hca_compress(x, lens, Wm, beta, m=s["m"], out=out)
+        ev[i][1].record()
+    torch.cuda.synchronize()
+    csa.check_device_error()
+    ms = statistics.median(a.elapsed_time(b) for a, b in ev)
+    byts = 2 * (x.numel() + out.numel())
+    return {"us": 1000 * ms, "tokens": int(s["B"] * s["n"]), "bytes": byts,
+            "achieved_gbs": byts / (ms * 1e-3) / 1e9, "frac_of_measured_hbm": byts / (ms * 1e-3) / 1e9 / hbm}
 
 
 # --------------------------------------------------------------------------
@@ -315,6 +493,9 @@ def main():
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if args.gpus != world and world > 1:
         print(f"warning: --gpus {args.gpus} but WORLD_SIZE={world}", file=sys.stderr)
+
+    if args.workload != 4 and args.impl == "ours":
+        return run_other_workload(args) if rank == 0 else 0
 
     if args.impl == "reference":
         if rank != 0:

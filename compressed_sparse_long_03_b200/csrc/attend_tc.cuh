@@ -35,7 +35,7 @@
 
 namespace csa {
 
-constexpr int kAtThreads = 128;
+constexpr int kAtThreads = 256;  // two threads per TMEM lane (head): column halves
 constexpr int kAtMaxTile = 192;                      // keys per tile
 constexpr uint32_t kAtQAtom = 128 * 128;             // 128 rows x 128 B
 constexpr uint32_t kAtKHalf = kAtMaxTile * 128;      // one 64-wide d slice of the key tile
@@ -54,6 +54,7 @@ __global__ void __launch_bounds__(kAtThreads, 1) k_attend_tc(AttendArgs a) {
   __shared__ int kvalid[kAtMaxTile / 32];  // validity bits, one word per 32 keys
   __shared__ const __nv_bfloat16 *rowp[kAtMaxTile];
   __shared__ float pm[136], pl[136];   // pushed partial max / sum [hl * CS + c]
+  __shared__ float xmax[2][128];       // per-half row max (then sum) of the partner
   __shared__ float mw[136], minv[128];  // merge weights [hl * CS + c], 1 / sum
   __shared__ int abort_flag;
 
@@ -76,8 +77,27 @@ __global__ void __launch_bounds__(kAtThreads, 1) k_attend_tc(AttendArgs a) {
   const __nv_bfloat16 *kv_tok = static_cast<const __nv_bfloat16 *>(a.kv_tok);
   __nv_bfloat16 *out = static_cast<__nv_bfloat16 *>(a.out) + (size_t)r * H * D;
 
+  // set-up that touches no global memory runs before the wait on the
+  // previous kernel: barriers and the TMEM allocation
+  if (warp == 0) {
+    tmem_alloc(smem_u32(&tmem_holder), 512);
+    tmem_relinquish();
+  }
+  if (tid == 0) {
+    abort_flag = 0;
+    mbar_init(smem_u32(&bar_s), 1);
+    mbar_init(smem_u32(&bar_o), 1);
+    fence_barrier_init();
+  }
   pdl_wait();
   pdl_launch_dependents();
+  // Q rows (heads) in the swizzled K-major layout; heads >= H are zero rows
+  const __nv_bfloat16 *qrow = q + (size_t)r * H * D;
+  for (int u = tid; u < 128 * 16; u += kAtThreads) {
+    const int h = u >> 4, c = u & 15;
+    const uint32_t dst = smem_u32(sQ) + (c >> 3) * kAtQAtom + h * 128 + (((c & 7) ^ (h & 7)) << 4);
+    cp_async16(dst, h < H ? qrow + (size_t)h * D + c * 8 : qrow, h < H ? 16u : 0u);
+  }
   int t;
   bool ok = query_position(a.lens, a.q_pos, b, a.Tq, tq, t);
   int v = 0, w0 = 0, nwin = 0;
@@ -96,6 +116,13 @@ __global__ void __launch_bounds__(kAtThreads, 1) k_attend_tc(AttendArgs a) {
   if (!ok) {  // uniform over the cluster
     for (int u = tid; u < H * D; u += kAtThreads)
       if ((u / D) % CS == rank) out[u] = __float2bfloat16_rn(0.f);
+    cp_async_wait_all();
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+      tc_fence_after();
+      tmem_dealloc(tmem_holder, 512);
+    }
     return;
   }
 
@@ -103,35 +130,23 @@ __global__ void __launch_bounds__(kAtThreads, 1) k_attend_tc(AttendArgs a) {
   const int L = nsel + nwin;
   const int per = (L + CS - 1) / CS;
   const int lo = min(L, rank * per), hi = min(L, lo + per);
-
-  if (warp == 0) {
-    tmem_alloc(smem_u32(&tmem_holder), 512);
-    tmem_relinquish();
-  }
-  if (tid == 0) {
-    abort_flag = 0;
-    mbar_init(smem_u32(&bar_s), 1);
-    mbar_init(smem_u32(&bar_o), 1);
-    fence_barrier_init();
-  }
-  // Q rows (heads) in the swizzled K-major layout; heads >= H are zero rows
-  const __nv_bfloat16 *qrow = q + (size_t)r * H * D;
-  for (int u = tid; u < 128 * 16; u += kAtThreads) {
-    const int h = u >> 4, c = u & 15;
-    const uint32_t dst = smem_u32(sQ) + (c >> 3) * kAtQAtom + h * 128 + (((c & 7) ^ (h & 7)) << 4);
-    cp_async16(dst, h < H ? qrow + (size_t)h * D + c * 8 : qrow, h < H ? 16u : 0u);
-  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tS = tmem_holder, tO = tmem_holder + 256;
-  const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+  // warp w reads TMEM lanes 32*(w%4).. (its quadrant: heads hq..hq+31) and
+  // works on one half of the columns (w/4): the key chunks [c0, c1) of S and
+  // the output columns [64*half, 64*half+64) of O
+  const int quad = warp & 3, half = warp >> 2;
+  const int hrow = quad * 32 + (tid & 31);  // this thread's head (TMEM lane)
+  const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+  const bool live = quad * 32 < H;  // quadrants of padded heads (>= H) skip the math
   volatile int *abort = &abort_flag;
 
-  float o[D];
+  float o[D / 2];
 #pragma unroll
-  for (int e = 0; e < D; ++e) o[e] = 0.f;
-  float m_run = -INFINITY, l_run = 0.f;
+  for (int e = 0; e < D / 2; ++e) o[e] = 0.f;
+  float m_run = -INFINITY, l_run = 0.f;  // l_run: this half's share of the sum
   uint32_t ns = 0, no = 0;
   bool alive = true;
 
@@ -186,44 +201,67 @@ __global__ void __launch_bounds__(kAtThreads, 1) k_attend_tc(AttendArgs a) {
     ++ns;
     if (!alive) break;
     tc_fence_after();
-    // ---- softmax over this lane's (head's) row
+    // ---- softmax over this head's row, the two column halves in parallel:
+    // this thread's chunks are read from TMEM once (one wait), the row max
+    // is combined with the partner thread through shared memory
+    const int cs0 = (nchunk + 1) >> 1;
+    const int c0 = half ? cs0 : 0, c1 = half ? nchunk : cs0;
+    uint32_t sv[kAtMaxTile / 64][32];
     float mt = -INFINITY;
-    for (int c = 0; c < nchunk; ++c) {
-      uint32_t sv[32];
-      tmem_ld16(tS + lane_off + 32 * c, sv);
-      tmem_ld16(tS + lane_off + 32 * c + 16, sv + 16);
-      tmem_wait_ld_regs<32>(sv);
-      const uint32_t vm = (uint32_t)kvalid[c];
+    if (live) {
 #pragma unroll
-      for (int jj = 0; jj < 32; ++jj)
-        if ((vm >> jj) & 1u) mt = fmaxf(mt, __uint_as_float(sv[jj]) * a.scale_log2);
+      for (int i = 0; i < kAtMaxTile / 64; ++i) {
+        if (c0 + i < c1) {
+          tmem_ld16(tS + lane_off + 32 * (c0 + i), sv[i]);
+          tmem_ld16(tS + lane_off + 32 * (c0 + i) + 16, sv[i] + 16);
+        }
+      }
+      tmem_wait_ld();
+#pragma unroll
+      for (int i = 0; i < kAtMaxTile / 64; ++i) {
+        if (c0 + i < c1) {
+#pragma unroll
+          for (int jj = 0; jj < 32; ++jj) asm volatile("" : "+r"(sv[i][jj]));
+          const uint32_t vm = (uint32_t)kvalid[c0 + i];
+#pragma unroll
+          for (int jj = 0; jj < 32; ++jj)
+            if ((vm >> jj) & 1u) mt = fmaxf(mt, __uint_as_float(sv[i][jj]) * a.scale_log2);
+        }
+      }
     }
+    xmax[half][hrow] = mt;
+    __syncthreads();
+    mt = fmaxf(mt, xmax[half ^ 1][hrow]);
     const float m_new = fmaxf(m_run, mt);
     const float alpha = (m_new == -INFINITY) ? 1.f : ex2(m_run - m_new);
     float lsum = 0.f;
-    for (int c = 0; c < nchunk; ++c) {
-      uint32_t sv[32];
-      tmem_ld16(tS + lane_off + 32 * c, sv);
-      tmem_ld16(tS + lane_off + 32 * c + 16, sv + 16);
-      tmem_wait_ld_regs<32>(sv);
-      const uint32_t vm = (uint32_t)kvalid[c];
+    if (live) {
 #pragma unroll
-      for (int g = 0; g < 4; ++g) {  // 8 keys -> one 16-byte chunk of P
-        uint32_t pk[4];
+      for (int i = 0; i < kAtMaxTile / 64; ++i) {
+        if (c0 + i < c1) {
+          const int c = c0 + i;
+          const uint32_t vm = (uint32_t)kvalid[c];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int j0 = 8 * g + 2 * e;
-          const float p0v = ((vm >> j0) & 1u) ? ex2(__uint_as_float(sv[j0]) * a.scale_log2 - m_new) : 0.f;
-          const float p1v = ((vm >> (j0 + 1)) & 1u) ? ex2(__uint_as_float(sv[j0 + 1]) * a.scale_log2 - m_new) : 0.f;
-          lsum += p0v + p1v;
-          __nv_bfloat162 pr = __floats2bfloat162_rn(p0v, p1v);
-          pk[e] = *reinterpret_cast<uint32_t *>(&pr);
+          for (int g = 0; g < 4; ++g) {  // 8 keys -> one 16-byte chunk of P
+            uint32_t pk[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int j0 = 8 * g + 2 * e;
+              const float p0v = ((vm >> j0) & 1u) ? ex2(__uint_as_float(sv[i][j0]) * a.scale_log2 - m_new) : 0.f;
+              const float p1v =
+                  ((vm >> (j0 + 1)) & 1u) ? ex2(__uint_as_float(sv[i][j0 + 1]) * a.scale_log2 - m_new) : 0.f;
+              lsum += p0v + p1v;
+              __nv_bfloat162 pr = __floats2bfloat162_rn(p0v, p1v);
+              pk[e] = *reinterpret_cast<uint32_t *>(&pr);
+            }
+            const int kg = 4 * c + g;  // 8-key group index 0..23
+            const uint32_t dst =
+                smem_u32(sP) + (kg >> 3) * kAtPAtom + hrow * 128 + (((kg & 7) ^ (hrow & 7)) << 4);
+            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(pk[0]), "r"(pk[1]),
+                         "r"(pk[2]), "r"(pk[3])
+                         : "memory");
+          }
         }
-        const int kg = 4 * c + g;  // 8-key group index 0..31
-        const uint32_t dst = smem_u32(sP) + (kg >> 3) * kAtPAtom + tid * 128 + (((kg & 7) ^ (tid & 7)) << 4);
-        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(pk[0]), "r"(pk[1]),
-                     "r"(pk[2]), "r"(pk[3])
-                     : "memory");
       }
     }
     if (m_new != -INFINITY) {
@@ -250,28 +288,33 @@ __global__ void __launch_bounds__(kAtThreads, 1) k_attend_tc(AttendArgs a) {
     if (!alive) break;
     tc_fence_after();
     const float scl = (m_new == -INFINITY) ? 1.f : alpha;
+    if (live) {
+      uint32_t ov[D / 2];
 #pragma unroll
-    for (int c = 0; c < D / 32; ++c) {
-      uint32_t ov[32];
-      tmem_ld16(tO + lane_off + 32 * c, ov);
-      tmem_ld16(tO + lane_off + 32 * c + 16, ov + 16);
-      tmem_wait_ld_regs<32>(ov);
+      for (int c = 0; c < D / 32; ++c) tmem_ld16(tO + lane_off + half * (D / 2) + 16 * c, ov + 16 * c);
+      tmem_wait_ld_regs<D / 2>(ov);
 #pragma unroll
-      for (int jj = 0; jj < 32; ++jj) o[32 * c + jj] = fmaf(o[32 * c + jj], scl, __uint_as_float(ov[jj]));
+      for (int e = 0; e < D / 2; ++e) o[e] = fmaf(o[e], scl, __uint_as_float(ov[e]));
     }
     tc_fence_before();
     __syncthreads();  // every lane done with S, P and O before they are rewritten
   }
 
   // ---- push this CTA's partial (max, sum, output) of head h into the CTA
-  // that finalises h (rank h % CS), one cluster barrier, merge locally
-  if (tid < H) {
-    const int own = tid % CS, slot = (tid / CS) * CS + rank;
-    float4 *dst = reinterpret_cast<float4 *>(att_peer<CS>(part, own) + (size_t)slot * D);
+  // that finalises h (rank h % CS), one cluster barrier, merge locally; the
+  // two halves of a row push their output columns, half 0 the max and the
+  // sum of both halves
+  xmax[half][hrow] = l_run;
+  __syncthreads();
+  if (hrow < H) {
+    const int own = hrow % CS, slot = (hrow / CS) * CS + rank;
+    float4 *dst = reinterpret_cast<float4 *>(att_peer<CS>(part, own) + (size_t)slot * D + half * (D / 2));
 #pragma unroll
-    for (int j = 0; j < D / 4; ++j) dst[j] = make_float4(o[4 * j], o[4 * j + 1], o[4 * j + 2], o[4 * j + 3]);
-    att_peer<CS>(pm, own)[slot] = m_run;
-    att_peer<CS>(pl, own)[slot] = l_run;
+    for (int j = 0; j < D / 8; ++j) dst[j] = make_float4(o[4 * j], o[4 * j + 1], o[4 * j + 2], o[4 * j + 3]);
+    if (half == 0) {
+      att_peer<CS>(pm, own)[slot] = m_run;
+      att_peer<CS>(pl, own)[slot] = l_run + xmax[1][hrow];
+    }
   }
   att_cluster_sync<CS>();
   // merge weights of this CTA's heads (h = rank + CS * hl), ranks in order

@@ -390,9 +390,10 @@ int launch_attend_fma(const csa::AttendArgs &a, int R, long max_keys, cudaStream
 // Tensor-core attention (bf16, d = 128): enough clusters to fill the GPU
 // when the batch is small, one CTA per row when rows alone fill it.
 int launch_attend_tc(const csa::AttendArgs &a, int R, cudaStream_t st, const char *what) {
-  const int want = (2 * num_sms() + R - 1) / R;
+  // one CTA per SM (its shared memory allows no second): the largest
+  // cluster, up to 8, that keeps all R * cs CTAs in one wave
   int cs = 1;
-  while (cs < 8 && cs < want) cs *= 2;
+  while (cs < 8 && (long)R * cs * 2 <= num_sms()) cs *= 2;
   void (*kern)(csa::AttendArgs) = nullptr;
   switch (cs) {
     case 1: kern = csa::k_attend_tc<1>; break;

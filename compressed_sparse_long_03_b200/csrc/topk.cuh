@@ -62,13 +62,14 @@ struct TopkShared {
   unsigned char all_cta[kTopkRankCap];
 };
 
-// Dynamic shared memory of one CTA for slices of up to `per` keys: the keys
-// (plus alignment slack), the candidates (key and position), two bit masks
-// over the slice (keys above the threshold bin, chosen candidates) and the
-// largest bin of every 32-key group.
+// Dynamic shared memory of one CTA for slices of up to `per` keys: two bit
+// masks over the slice (chosen candidates, keys above the threshold bin) and
+// the largest bin of every 32-key group, then the keys (plus alignment
+// slack), then the candidates (key and position).
+__host__ __device__ constexpr size_t topk_mask_words(int per) { return ((size_t)per + 3 + 31) / 32; }
 __host__ __device__ constexpr size_t topk_dyn_bytes(int per) {
-  return 4ull * ((size_t)per + 4 + 2 * (size_t)(per < kTopkRankCap ? per : kTopkRankCap) +
-                 3 * (((size_t)per + 3 + 31) / 32));
+  return 4ull * (((3 * topk_mask_words(per) + 3) & ~(size_t)3) + (size_t)per + 4 +
+                 2 * (size_t)(per < kTopkRankCap ? per : kTopkRankCap));
 }
 
 template <int CS>
@@ -120,6 +121,29 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(const float *__restrict__
   const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
   const unsigned lt = (1u << lane) - 1u;
   int32_t *orow = idx_out + (size_t)r * k;
+
+  // layout for the largest slice (the same in every CTA of the cluster, so
+  // peers find each other's candidates at the same offsets)
+  const int per_max = (nc_max + CS - 1) / CS;
+  const int nw_max = (int)topk_mask_words(per_max);
+  const int ccap = per_max < kTopkRankCap ? per_max : kTopkRankCap;
+  const int koff = (3 * nw_max + 3) & ~3;  // keys start 16-byte aligned
+  uint32_t *selbits = dyn;                                         // chosen candidates
+  uint32_t *abovebits = dyn + nw_max;                              // decided above b*
+  uint32_t *gmaxbin = dyn + 2 * nw_max;                            // largest bin of a group
+  uint32_t *cand_key = dyn + koff + per_max + 4;                   // [ccap]
+  int *cand_pos = reinterpret_cast<int *>(cand_key + ccap);        // [ccap]
+
+  // shared-memory set-up touches no global memory: before the wait
+  for (int j = tid; j < kScoreBins; j += NT) sh.hist[j] = 0;
+  if (tid < kTopkSuper) sh.super[tid] = 0;
+  if (tid == 0) {
+    sh.ncand = 0;
+    sh.above = 0;
+  }
+  if (tid < 16) sh.peer_sel[tid] = 0;
+  for (int j = tid; j < 3 * nw_max; j += NT) dyn[j] = 0u;  // both masks and group maxima
+  __syncthreads();
   pdl_wait();
   pdl_launch_dependents();
 
@@ -140,7 +164,6 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(const float *__restrict__
   const int per = (v + CS - 1) / CS;  // the same in every CTA of the cluster
   const int lo = min(v, rank * per), hi = min(v, lo + per);
   const int len = hi - lo;
-  const int ccap = per < kTopkRankCap ? per : kTopkRankCap;
   const float *srow = scores + (size_t)r * nc_max;
   // the slice start's misalignment to 16 B, mirrored in the key array so that
   // vector loads and vector stores line up.  Key j sits at position
@@ -148,24 +171,8 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(const float *__restrict__
   // never split a 16-byte vector.
   const int head0 = (int)((16 - (reinterpret_cast<uintptr_t>(srow + lo) & 15)) & 15) / 4;
   const int p0 = (4 - head0) & 3;
-  const int nwords = (per + 3 + 31) / 32;
   const int ngroups = (p0 + len + 31) / 32;
-  uint32_t *keys = dyn + p0;                                      // [per], keys+head0 16 B aligned
-  uint32_t *cand_key = dyn + per + 4;                             // [ccap]
-  int *cand_pos = reinterpret_cast<int *>(dyn + per + 4 + ccap);  // [ccap]
-  uint32_t *selbits = dyn + per + 4 + 2 * ccap;                   // [nwords] chosen candidates
-  uint32_t *abovebits = selbits + nwords;                         // [nwords] decided above b*
-  uint32_t *gmaxbin = abovebits + nwords;                         // [nwords] largest bin of a group
-
-  for (int j = tid; j < kScoreBins; j += NT) sh.hist[j] = 0;
-  if (tid < kTopkSuper) sh.super[tid] = 0;
-  if (tid == 0) {
-    sh.ncand = 0;
-    sh.above = 0;
-  }
-  if (tid < 16) sh.peer_sel[tid] = 0;
-  for (int j = tid; j < 3 * nwords; j += NT) selbits[j] = 0u;  // both masks and group maxima
-  __syncthreads();
+  uint32_t *keys = dyn + koff + p0;  // [per], keys+head0 16 B aligned
 
   // ---- A: keys (16-byte vector loads, eight in flight per thread) and the
   // local histogram of their 12 leading bits

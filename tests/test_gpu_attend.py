@@ -53,6 +53,29 @@ def test_csa_attend(dt, d, H, k, nc, window, n_tok):
     assert_close(to_host(out), ref, dt, "csa_attend")
 
 
+@pytest.mark.parametrize("H,B,Tq", [
+    (4, 1, 2),      # 2 rows: 8-CTA clusters, fewer heads than CTAs (owners without heads)
+    (100, 1, 37),   # 37 rows: 4-CTA clusters, a partly padded TMEM lane quadrant
+    (128, 2, 37),   # 74 rows: 2-CTA clusters, every lane a head
+    (64, 2, 150),   # 300 rows: one CTA per row, two key tiles per CTA
+])
+def test_csa_attend_cluster_shapes(H, B, Tq):
+    """The tensor-core attention at every cluster size it launches with and at
+    head counts that leave owners without heads or pad a lane quadrant."""
+    seed = 900 + H + Tq
+    d, k, nc, window, n_tok = 128, 256, 2000, 128, 8192
+    lens = np.array([4 * nc, 4 * nc - 77][:B], np.int32)
+    q = W.normal(seed, "q", (B, Tq, H, d), 1.0, "bf16")
+    kv = W.normal(seed, "kv", (B, nc, d), 1.0, "bf16")
+    tok = W.normal(seed, "win", (B, n_tok, d), 1.0, "bf16")
+    vis = oracle.visible(lens, B, Tq, 4)
+    idx = random_idx(seed, B, Tq, k, vis, nc)
+    out = csa.csa_attend(to_dev(q), to_dev(kv), to_dev(tok), to_dev(idx), to_dev(lens), window=window)
+    csa.check_device_error()
+    ref = oracle.attend(q, kv, tok, lens, idx=idx, window=window)
+    assert_close(to_host(out), ref, "bf16", "csa_attend")
+
+
 @pytest.mark.parametrize("dt,d,H,m", [("bf16", 128, 64, 128), ("f32", 64, 8, 8), ("bf16", 128, 16, 4)])
 def test_hca_attend_ragged(dt, d, H, m):
     seed = 3 * m + H
