@@ -11,6 +11,7 @@
 #include <cstdio>
 #include <cstring>
 #include <algorithm>
+#include <type_traits>
 #include <mutex>
 #include <string>
 #include <unordered_map>
@@ -20,6 +21,7 @@
 
 #include "common.cuh"
 #include "compress.cuh"
+#include "compress_tc.cuh"
 #include "index_score_fma.cuh"
 #include "index_score_tc.cuh"
 #include "topk.cuh"
@@ -220,10 +222,55 @@ int attend_cluster_size(long max_keys) {
 // ---------------------------------------------------------------------------
 // compressors
 // ---------------------------------------------------------------------------
+// bf16 compressors with d in {64, 128} (HCA: strides that keep 32-token
+// chunks inside one entry) run on the tensor cores.
+template <bool CSA, int D>
+int launch_compress_tc(const void *x, const int32_t *lens, int B, int n_max, int m, const void *Wa,
+                       const void *Wb, const void *bias, void *out, int nc_max, cudaStream_t st,
+                       const char *what) {
+  constexpr int NTOK = CSA ? 128 + csa::kCtHalo : 128;
+  constexpr size_t A_SER = (size_t)(D / 64) * 128 * 128, X_STAGE = (size_t)(D / 64) * NTOK * 128;
+  constexpr int NSER = CSA ? 2 : 1, NB = CSA ? 1 : 2;
+  if (nc_max == 0 || B == 0) return CSA_OK;
+  CUtensorMap tmX;
+  int rc = encode_bf16_2d(&tmX, x, D, (uint64_t)B * n_max, 64, NTOK, what);
+  if (rc) return rc;
+  // the token stages also hold W while it is transposed
+  const size_t budget = 227 * 1024 - 1024 - NSER * A_SER - 4096;
+  const int stages = (int)std::min<size_t>(5, budget / X_STAGE);
+  if ((size_t)stages * X_STAGE < NSER * (size_t)D * D * 2)
+    return fail(CSA_ERR_UNSUPPORTED, "%s: shared memory too small", what);
+  const size_t smem = 1024 + NSER * A_SER + stages * X_STAGE + 8 * (2 * stages + 2 * NB + 1);
+  auto kern = csa::k_compress_tc<CSA, D>;
+  rc = ensure_smem(kern, smem, what);
+  if (rc) return rc;
+  csa::CompressTcArgs a;
+  a.Wa = static_cast<const __nv_bfloat16 *>(Wa);
+  a.Wb = static_cast<const __nv_bfloat16 *>(Wb);
+  a.bias = static_cast<const __nv_bfloat16 *>(bias);
+  a.lens = lens;
+  a.out = static_cast<__nv_bfloat16 *>(out);
+  a.n_max = n_max;
+  a.nc_max = nc_max;
+  a.m = m;
+  if (CSA) a.per_seq = (nc_max + 31) / 32;
+  else if (m > 128) a.per_seq = nc_max;
+  else a.per_seq = (int)(((long)nc_max * m + 127) / 128);
+  a.units = B * a.per_seq;
+  a.stages = stages;
+  const unsigned grid = (unsigned)std::min(a.units, num_sms());
+  return launch_cluster(kern, 1, grid, csa::kCtThreads, smem, st, what, tmX, a);
+}
+
 template <typename T>
 int launch_csa_compress(const void *x, const int32_t *lens, int B, int n_max, int d, const void *Wa,
                         const void *Wb, const void *b8, void *out, cudaStream_t st) {
   const int nc_max = (n_max + 3) / 4;
+  const bool tc_rows_ok = (long)B * n_max < (1L << 30);  // TMA row coordinates fit in int32
+  if constexpr (std::is_same<T, __nv_bfloat16>::value) {
+    if (d == 64 && tc_rows_ok) return launch_compress_tc<true, 64>(x, lens, B, n_max, 4, Wa, Wb, b8, out, nc_max, st, "csa_compress");
+    if (d == 128 && tc_rows_ok) return launch_compress_tc<true, 128>(x, lens, B, n_max, 4, Wa, Wb, b8, out, nc_max, st, "csa_compress");
+  }
   dim3 grid((nc_max + csa::kCsaEntries - 1) / csa::kCsaEntries, B);
   auto X = static_cast<const T *>(x);
   auto A = static_cast<const T *>(Wa);
@@ -243,6 +290,13 @@ template <typename T>
 int launch_hca_compress(const void *x, const int32_t *lens, int B, int n_max, int d, int m,
                         const void *W, const void *bias, void *out, cudaStream_t st) {
   const int nc_max = (int)(((long)n_max + m - 1) / m);
+  const bool tc_ok = csa::hca_tc_stride_ok(m) && (long)B * n_max < (1L << 30);
+  if constexpr (std::is_same<T, __nv_bfloat16>::value) {
+    if (tc_ok && d == 64)
+      return launch_compress_tc<false, 64>(x, lens, B, n_max, m, W, nullptr, bias, out, nc_max, st, "hca_compress");
+    if (tc_ok && d == 128)
+      return launch_compress_tc<false, 128>(x, lens, B, n_max, m, W, nullptr, bias, out, nc_max, st, "hca_compress");
+  }
   dim3 grid(nc_max, B);
   auto X = static_cast<const T *>(x);
   auto Wp = static_cast<const T *>(W);

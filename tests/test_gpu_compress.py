@@ -37,6 +37,17 @@ def test_csa_compress_ragged(dt, d, std):
             np.all(got[b, (lens[b] + 3) // 4:] == 0)
 
 
+@pytest.mark.parametrize("d", [64, 128])
+def test_csa_compress_many_tiles_per_cta(d):
+    """More 32-entry tiles than CTAs (each CTA loops), ragged tails."""
+    B, n_max = 8, 20000
+    lens = [20000, 19999, 16385, 4097, 128, 3, 1, 12345]
+    x, lens, Wa, Wb, beta = _csa_case("bf16", d, B, n_max, lens, 77 + d, d ** -0.5)
+    out = csa.csa_compress(to_dev(x), to_dev(lens), to_dev(Wa), to_dev(Wb), to_dev(beta))
+    ref = oracle.csa_compress(x, lens, Wa, Wb, beta)
+    assert_close(to_host(out), ref, "bf16", "csa_compress")
+
+
 def test_csa_compress_full_prefill_workload():
     """Workload 2 (bf16, 8192 tokens, d=128): both the KV cache and the
     indexer-key cache, every row."""
@@ -48,7 +59,9 @@ def test_csa_compress_full_prefill_workload():
         assert_close(to_host(out), ref, "bf16", f"csa_compress({xk})")
 
 
-@pytest.mark.parametrize("dt,m,d", [("f32", 8, 64), ("bf16", 128, 128), ("bf16", 100, 64), ("f32", 1, 32)])
+@pytest.mark.parametrize("dt,m,d", [("f32", 8, 64), ("bf16", 128, 128), ("bf16", 100, 64), ("f32", 1, 32),
+                                    ("bf16", 32, 128), ("bf16", 64, 64), ("bf16", 256, 128),
+                                    ("bf16", 384, 64)])
 def test_hca_compress_ragged(dt, m, d):
     B, n_max = 3, 5 * m + 13
     seed = 40 + m
