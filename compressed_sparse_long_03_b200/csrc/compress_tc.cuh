@@ -41,6 +41,8 @@
 // All waits are time-bounded (sm100.cuh).
 #pragma once
 
+#include <type_traits>
+
 #include "common.cuh"
 #include "sm100.cuh"
 
@@ -258,9 +260,12 @@ __global__ void __launch_bounds__(kCtThreads, 1)
     bool alive = true;
     // HCA online state of the current entry (this half's tokens)
     float run_max = -INFINITY, den = 0.f, num = 0.f;
+    // the next unit's sequence length is loaded one unit ahead
+    int n_next = blockIdx.x < a.units ? __ldg(a.lens + blockIdx.x / a.per_seq) : 0;
     for (int u = blockIdx.x; u < a.units && alive; u += gridDim.x) {
       const int b = u / a.per_seq, t = u % a.per_seq;
-      int n = __ldg(a.lens + b);
+      int n = n_next;
+      if (u + (int)gridDim.x < a.units) n_next = __ldg(a.lens + (u + (int)gridDim.x) / a.per_seq);
       if (n < 0 || n > a.n_max) {
         if (t == 0 && c == 0 && half == 0) raise_dev_err(kDevErrLen);
         n = 0;
@@ -324,67 +329,89 @@ __global__ void __launch_bounds__(kCtThreads, 1)
         } else {
           const int m = a.m;
           const long tok0 = (m > 128) ? (long)m * t + 128L * jt : 128L * t;
-#pragma unroll 1
-          for (int ch = 2 * half; ch < 2 * half + 2; ++ch) {  // 32-token chunks, each inside one entry
-            const int col0 = 32 * ch;
-            const long s0 = tok0 + col0;
-            const int i = (int)(s0 / m);               // the chunk's entry
-            const int pos0 = (int)(s0 - (long)m * i);  // its first token's slot in the entry
-            if (live) {
-              uint32_t zt[32];
-              tmem_ld16(tb + col0, zt);
-              tmem_ld16(tb + col0 + 16, zt + 16);
-              tmem_wait_ld_regs<32>(zt);
-              float z[32];
-              float cmax = -INFINITY;
-              const long lim = (long)n - s0;  // tokens of the chunk inside the sequence
-              if (m <= 128) {
-                uint32_t bt[32];
-                tmem_ld16(tmem + lane_off + BIAS_COL + pos0, bt);
-                tmem_ld16(tmem + lane_off + BIAS_COL + pos0 + 16, bt + 16);
-                tmem_wait_ld_regs<32>(bt);
+          const bool bias_tmem = m <= 128;  // warp-uniform
+          // fold G consecutive tokens (tile columns colL.., entry slots pos0..)
+          // of one entry into this thread's running (max, sum, pooled sum);
+          // lim = how many of them lie inside the sequence
+          auto fold = [&](auto Gc, int colL, int pos0, long lim) {
+            constexpr int G = decltype(Gc)::value;
+            constexpr int NCH = G / 8;  // independent chains
+            uint32_t zt[G], bt[G];
 #pragma unroll
-                for (int jj = 0; jj < 32; ++jj)
-                  z[jj] = fmaf(__uint_as_float(zt[jj]), kLog2e, __uint_as_float(bt[jj]));
-              } else {
-                const __nv_bfloat16 *bp = a.bias + (size_t)pos0 * D + c;
+            for (int q = 0; q < G / 16; ++q) tmem_ld16(tb + colL + 16 * q, zt + 16 * q);
+            if (bias_tmem) {
 #pragma unroll
-                for (int jj = 0; jj < 32; ++jj)
-                  z[jj] = (__uint_as_float(zt[jj]) + __bfloat162float(bp[jj * D])) * kLog2e;
-              }
-              if (lim < 32) {
-#pragma unroll
-                for (int jj = 0; jj < 32; ++jj)
-                  if (jj >= lim) z[jj] = -INFINITY;
-              }
-#pragma unroll
-              for (int jj = 0; jj < 32; ++jj) cmax = fmaxf(cmax, z[jj]);
-              const float nmax = fmaxf(run_max, cmax);
-              if (nmax != -INFINITY) {
-                const float alpha = ex2(run_max - nmax);  // 0 when run_max is -inf
-                den *= alpha;
-                num *= alpha;
-                // chunk rows start at a multiple of 32: row % 8 == jj % 8
-                const uint8_t *rb = sX + s * X_STAGE + col0 * 128;
-#pragma unroll
-                for (int jj = 0; jj < 32; ++jj) {
-                  const float pw = ex2(z[jj] - nmax);  // 0 for masked tokens
-                  den += pw;
-                  num = fmaf(pw, xat(rb + jj * 128, jj & 7), num);
-                }
-                run_max = nmax;
-              }
+              for (int q = 0; q < G / 16; ++q) tmem_ld16(tmem + lane_off + BIAS_COL + pos0 + 16 * q, bt + 16 * q);
             }
-            if (m <= 64) {
-              // the entry lies in this half: it ends with this chunk or the next
-              if (pos0 + 32 == m) {
-                if (live && i < a.nc_max)
-                  a.out[((size_t)b * a.nc_max + i) * D + c] = __float2bfloat16_rn(den > 0.f ? num / den : 0.f);
-                run_max = -INFINITY;
-                den = 0.f;
-                num = 0.f;
-              }
-            } else if (ch == 2 * half + 1 && pos0 + 32 + (1 - half) * 64 == m) {
+            tmem_wait_ld_regs<G>(zt);
+            float z[G];
+            if (bias_tmem) {
+              tmem_wait_ld_regs<G>(bt);
+#pragma unroll
+              for (int jj = 0; jj < G; ++jj) z[jj] = fmaf(__uint_as_float(zt[jj]), kLog2e, __uint_as_float(bt[jj]));
+            } else {
+              const __nv_bfloat16 *bp = a.bias + (size_t)pos0 * D + c;
+#pragma unroll
+              for (int jj = 0; jj < G; ++jj)
+                z[jj] = (__uint_as_float(zt[jj]) + __bfloat162float(bp[jj * D])) * kLog2e;
+            }
+            if (lim < G) {
+#pragma unroll
+              for (int jj = 0; jj < G; ++jj)
+                if (jj >= lim) z[jj] = -INFINITY;
+            }
+            float cm[NCH];
+#pragma unroll
+            for (int k = 0; k < NCH; ++k) cm[k] = -INFINITY;
+#pragma unroll
+            for (int jj = 0; jj < G; ++jj) cm[jj % NCH] = fmaxf(cm[jj % NCH], z[jj]);
+#pragma unroll
+            for (int k = 1; k < NCH; ++k) cm[0] = fmaxf(cm[0], cm[k]);
+            const float nmax = fmaxf(run_max, cm[0]);
+            if (nmax == -INFINITY) return;
+            const float alpha = ex2(run_max - nmax);  // 0 when run_max is -inf
+            // rows colL.. start at a multiple of 32: row % 8 == jj % 8
+            const uint8_t *rb = sX + s * X_STAGE + colL * 128;
+            float dd[NCH], nn[NCH];
+#pragma unroll
+            for (int k = 0; k < NCH; ++k) dd[k] = nn[k] = 0.f;
+#pragma unroll
+            for (int jj = 0; jj < G; ++jj) {
+              const float pw = ex2(z[jj] - nmax);  // 0 for masked tokens
+              dd[jj % NCH] += pw;
+              nn[jj % NCH] = fmaf(pw, xat(rb + jj * 128, jj & 7), nn[jj % NCH]);
+            }
+#pragma unroll
+            for (int k = 1; k < NCH; ++k) {
+              dd[0] += dd[k];
+              nn[0] += nn[k];
+            }
+            den = fmaf(den, alpha, dd[0]);
+            num = fmaf(num, alpha, nn[0]);
+            run_max = nmax;
+          };
+          auto finish = [&](int i) {
+            if (live && i < a.nc_max)
+              a.out[((size_t)b * a.nc_max + i) * D + c] = __float2bfloat16_rn(den > 0.f ? num / den : 0.f);
+            run_max = -INFINITY;
+            den = 0.f;
+            num = 0.f;
+          };
+          if (m == 32) {  // two entries per half, one chunk each
+#pragma unroll 1
+            for (int ch = 2 * half; ch < 2 * half + 2; ++ch) {
+              const long s0 = tok0 + 32 * ch;
+              if (live) fold(std::integral_constant<int, 32>(), 32 * ch, 0, (long)n - s0);
+              finish((int)(s0 / 32));
+            }
+          } else {  // the half's 64 tokens lie inside one entry
+            const long s0 = tok0 + 64 * half;
+            const int i = (int)(s0 / m);
+            const int pos0 = (int)(s0 - (long)m * i);
+            if (live) fold(std::integral_constant<int, 64>(), 64 * half, pos0, (long)n - s0);
+            if (m == 64) {
+              finish(i);
+            } else if (pos0 + 64 + (1 - half) * 64 == m) {
               // the entry (both halves) ends with this tile: merge below
               merge = true;
               merge_i = i;
