@@ -249,33 +249,78 @@ def run_ours(args, rank, world, dev):
     csa.check_device_error()
     ms = t0.elapsed_time(t1) / K
 
-    # end to end through the public API from pinned host buffers: one H2D
-    # copy of the step's query inputs (q, q_I, w packed), the two calls, one
-    # D2H copy of the output
+    # end to end through the public API from pinned host buffers, as a
+    # serving loop runs it: every step copies its query-side inputs (q, q_I,
+    # w packed: one H2D copy) in and its output (one D2H copy) out; the
+    # inputs and outputs are double-buffered, the copies run on two copy
+    # streams, so step i+1's upload and step i's download overlap step i's
+    # kernels.  The timed region covers every step's copies.
     host = torch.from_numpy(np.concatenate([np.ascontiguousarray(wl[n]).reshape(-1).view(np.int16)
                                             for n in qnames])).pin_memory()
-    out_h = torch.empty(out.shape, dtype=torch.bfloat16).pin_memory()
+    packs = [pack, torch.empty_like(pack)]
+    views = []
+    for pk in packs:
+        o, vw = 0, {}
+        for n in qnames:
+            sz = D[n].numel()
+            vw[n] = pk[o:o + sz].view(D[n].shape)
+            o += sz
+        views.append(vw)
+    outs = [out, torch.empty_like(out)]
+    outs_h = [torch.empty(out.shape, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+    up, down = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+    in_ready, pack_free, out_ready, out_free = ([torch.cuda.Event(), torch.cuda.Event()]
+                                                for _ in range(4))
 
-    def step_e2e():
-        pack.view(torch.int16).copy_(host, non_blocking=True)
-        step()
-        out_h.copy_(out, non_blocking=True)
+    def upload(i):
+        j = i % 2
+        with torch.cuda.stream(up):
+            if i >= 2:
+                up.wait_event(pack_free[j])      # step i-2 no longer reads this pack
+            packs[j].view(torch.int16).copy_(host, non_blocking=True)
+            in_ready[j].record(up)
+
+    def compute_and_download(i):
+        j = i % 2
+        stream.wait_event(in_ready[j])
+        if i >= 2:
+            stream.wait_event(out_free[j])       # step i-2's output has been read out
+        vw = views[j]
+        csa.csa_index_topk(vw["qI"], vw["w"], D["kI"], D["lens"], k, idx_out=idx, workspace=ws)
+        csa.csa_attend(vw["q"], D["kv"], D["win"], idx, D["lens"], window=window, out=outs[j])
+        pack_free[j].record(stream)
+        out_ready[j].record(stream)
+        with torch.cuda.stream(down):
+            down.wait_event(out_ready[j])
+            outs_h[j].copy_(outs[j], non_blocking=True)
+            out_free[j].record(down)
+
+    def run_e2e(n_steps, start):
+        up.wait_event(start)  # no copy before the region opens
+        upload(0)
+        for i in range(n_steps):
+            if i + 1 < n_steps:
+                upload(i + 1)
+            compute_and_download(i)
+        stream.wait_event(out_free[(n_steps - 1) % 2])  # the last download is inside the region
 
     h2d = host.numel() * 2
-    d2h = out_h.numel() * 2
-    for _ in range(3):
-        step_e2e()
+    d2h = outs_h[0].numel() * 2
+    warm = torch.cuda.Event()
+    warm.record(stream)
+    run_e2e(4, warm)
+    torch.cuda.synchronize()
     Ke = max(10, K // 2)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
     torch.cuda.synchronize()
     e0.record(stream)
-    for _ in range(Ke):
-        step_e2e()
+    run_e2e(Ke, e0)
     e1.record(stream)
     torch.cuda.synchronize()
     barrier()
     ms_e2e = e0.elapsed_time(e1) / Ke
+    csa.check_device_error()
 
     ms, ms_e2e = max_over_ranks([ms, ms_e2e], world, f"cuda:{dev}")
     return dict(ms=ms, ms_e2e=ms_e2e, stage=stage, clocks=clocks, s=s, B=B, h2d=h2d, d2h=d2h,

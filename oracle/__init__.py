@@ -53,7 +53,7 @@ def _load():
         lib.orc_index_scores.argtypes = [P, P, P, P, P, I, I, I, I, I, I, P]
         lib.orc_select_topk.argtypes = [P, P, L, I, I, P]
         lib.orc_visible.argtypes = [P, P, I, I, I, P]
-        lib.orc_attend.argtypes = [P, P, P, I, P, P, P, I, I, I, I, I, I, I, I, D, I, P]
+        lib.orc_attend.argtypes = [P, P, P, I, P, P, P, I, I, I, I, I, I, I, I, D, P, I, P]
         lib.orc_set_threads.argtypes = [I]
         lib.orc_get_threads.restype = I
         for name in ("orc_round", "orc_csa_compress", "orc_hca_compress", "orc_index_scores",
@@ -207,10 +207,10 @@ def index_topk(qI, w, kI, lens, k, q_pos=None):
     return select_topk(sc, vis, k), sc
 
 
-def attend(q, kv_c, kv_tok, lens, idx=None, q_pos=None, window=128, m=4, scale=0.0):
+def attend(q, kv_c, kv_tok, lens, idx=None, q_pos=None, window=128, m=4, scale=0.0, sink=None):
     """a5 (idx given, CSA) / a6 (idx None, HCA with stride m): q [B][Tq][H][d],
-    kv_c [B][nc_max][d], kv_tok [B][n_tok][d] (ring: token s at row s % n_tok)
-    -> float64 [B][Tq][H][d]."""
+    kv_c [B][nc_max][d], kv_tok [B][n_tok][d] (ring: token s at row s % n_tok),
+    sink [H] per-head sink logits or None -> float64 [B][Tq][H][d]."""
     lib = _load()
     arrs = [q, kv_tok] + ([kv_c] if kv_c is not None and kv_c.size else [])
     dt = _same_dt(*arrs)
@@ -230,8 +230,11 @@ def attend(q, kv_c, kv_tok, lens, idx=None, q_pos=None, window=128, m=4, scale=0
     pp = None
     if q_pos is not None:
         q_pos, pp = _c(q_pos, np.int32)
+    ps = None
+    if sink is not None:
+        sink, ps = _c(np.asarray(sink, np.float64).reshape(H), np.float64)
     out = np.empty((B, Tq, H, d), np.float64)
     _check(lib.orc_attend(pq, pc if nc_max else None, pt, n_tok, pi, pl, pp, B, Tq, H, d,
-                          nc_max, k, window, m, float(scale), dt,
+                          nc_max, k, window, m, float(scale), ps, dt,
                           out.ctypes.data_as(ctypes.c_void_p)), "attend")
     return out

@@ -404,13 +404,19 @@ int orc_visible(const int32_t *lens, const int32_t *q_pos, int B, int Tq, int m,
  * visible entry (HCA).  The window token at position s is row (s mod n_tok)
  * of kv_tok[b] (a ring: it must hold the query's whole window,
  * min(W, t+1) <= n_tok).  scale <= 0 means 1/sqrt(d).
+ * [A4] second of the "three details": an attention sink, a learned logit
+ * per head whose exponential is added to the softmax denominator (so a
+ * head's weights may sum to less than one).  Reading: sink[h] is in the
+ * units of the scaled logits l and carries no value:
+ *   o[t,h] = sum_j e^{l_j} v_j / (sum_j e^{l_j} + e^{sink[h]});
+ * sink == NULL means no sink.
  * q: [B][Tq][H][d], kv_c: [B][nc_max][d], kv_tok: [B][n_tok][d],
- * idx: [B][Tq][k], out: [B][Tq][H][d] (double).
+ * idx: [B][Tq][k], sink: [H] (double), out: [B][Tq][H][d] (double).
  */
 int orc_attend(const void *q, const void *kv_c, const void *kv_tok, int n_tok,
                const int32_t *idx, const int32_t *lens, const int32_t *q_pos, int B, int Tq,
-               int H, int d, int nc_max, int k, int window, int m, double scale, int dt,
-               double *out) {
+               int H, int d, int nc_max, int k, int window, int m, double scale,
+               const double *sink, int dt, double *out) {
   if (!q || !kv_tok || !lens || !out) return ORC_ERR_ARG;
   if (B < 0 || Tq < 0 || H <= 0 || d <= 0 || nc_max < 0 || window <= 0 || m <= 0) return ORC_ERR_ARG;
   if (n_tok <= 0 || (idx && k <= 0) || (nc_max > 0 && !kv_c)) return ORC_ERR_ARG;
@@ -469,11 +475,13 @@ int orc_attend(const void *q, const void *kv_c, const void *kv_tok, int n_tok,
         lg[j] = scale * dot;
         if (lg[j] > mx) mx = lg[j];
       }
+      if (sink && sink[h] > mx) mx = sink[h];
       double den = 0.0;
       for (long j = 0; j < nk; ++j) {
         lg[j] = exp(lg[j] - mx);
         den += lg[j];
       }
+      if (sink) den += exp(sink[h] - mx);
       for (int e = 0; e < d; ++e) {
         double acc = 0.0;
         for (long j = 0; j < nk; ++j) acc += lg[j] * keys[j * d + e];

@@ -175,3 +175,50 @@ def test_bad_position_and_short_ring_are_errors():
         oracle.attend(q, kv, tok, lens, idx=None, window=17)
     with pytest.raises(oracle.OracleError):
         oracle.attend(q, kv, tok, lens, idx=None, window=8, q_pos=np.full((2, 2), 60, np.int32))
+
+
+# ---------------------------------------------------------------------------
+# attention sink: "Anatomy of a Frontier Model", second of the "three
+# details" (a learned per-head logit whose exponential joins the softmax
+# denominator)
+# ---------------------------------------------------------------------------
+def test_sink_single_key_is_logistic_weight():
+    """One key (query at t = 0: its own token, no entries): the output is the
+    key times the logistic function of (logit - sink)."""
+    q, kv, tok, lens = setup(seed=21)
+    H, d = q.shape[2], q.shape[3]
+    sink = np.array([-1.5, 0.0, 2.25])
+    q_pos = np.zeros((2, 2), np.int32)
+    out = oracle.attend(q, kv, tok, lens, idx=np.full((2, 2, 3), -1, np.int32), q_pos=q_pos, sink=sink)
+    for b in range(2):
+        for tq in range(2):
+            v = tok[b, 0].astype(np.float64)
+            for h in range(H):
+                logit = float(q[b, tq, h].astype(np.float64) @ v) / np.sqrt(d)
+                wgt = 1.0 / (1.0 + np.exp(sink[h] - logit))
+                np.testing.assert_allclose(out[b, tq, h], wgt * v, rtol=1e-13, atol=1e-14)
+
+
+def test_sink_limits():
+    """A sink of -1e300 changes nothing; a sink far above every logit drives
+    every output to zero."""
+    q, kv, tok, lens = setup(seed=22)
+    idx = np.array([[[0, 2, 5], [1, -1, 3]], [[4, 4, 0], [2, 7, 9]]], np.int32)
+    base = oracle.attend(q, kv, tok, lens, idx=idx)
+    low = oracle.attend(q, kv, tok, lens, idx=idx, sink=np.full(3, -1e300))
+    np.testing.assert_array_equal(low, base)
+    high = oracle.attend(q, kv, tok, lens, idx=idx, sink=np.full(3, 800.0))
+    assert np.abs(high).max() < 1e-300
+
+
+def test_sink_rescales_without_turning():
+    """With a sink each head's output is the sink-free output times one
+    factor in (0, 1): the sink carries no value, it only takes weight."""
+    q, kv, tok, lens = setup(seed=23, d=16)
+    idx = np.array([[[0, 2, 5], [1, -1, 3]], [[4, 4, 0], [2, 7, 9]]], np.int32)
+    base = oracle.attend(q, kv, tok, lens, idx=idx)
+    sunk = oracle.attend(q, kv, tok, lens, idx=idx, sink=np.array([0.3, -0.7, 1.1]))
+    ratio = sunk / base
+    spread = ratio.max(axis=-1) - ratio.min(axis=-1)
+    assert spread.max() < 1e-12
+    assert (ratio > 0).all() and (ratio < 1).all()

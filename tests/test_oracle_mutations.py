@@ -40,6 +40,7 @@ MUTANTS = {
     "attend_window_off_by_one": ("long w0 = t - window + 1;", "long w0 = t - window + 2;"),
     "attend_visibility": ("long vis = (t + 1) / m;", "long vis = (t + 2) / m;"),
     "attend_invisible_index_used": ("if (i < 0 || i >= vis) continue;", "if (i < 0 || i >= nc_max) continue;"),
+    "attend_sink_ignored": ("if (sink) den += exp(sink[h] - mx);", ""),
     "round_double_rounding": ("r = nearbyint(ldexp(a, -q));", "r = nearbyint(ldexp((double)(float)a, -q));"),
 }
 
