@@ -426,6 +426,20 @@ def run_other_workload(args):
         step()
     torch.cuda.synchronize()
     csa.check_device_error()
+    # the step is replayed from a CUDA graph, so that the GPU time of a step
+    # of small kernels is not the host's time to issue them
+    run, how = step, "issued eagerly"
+    try:
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            step()
+        graph.replay()
+        torch.cuda.synchronize()
+        csa.check_device_error()
+        run, how = graph.replay, "replayed from a CUDA graph"
+    except Exception as e:  # capture unsupported here: time the eager calls
+        how = f"issued eagerly (graph capture failed: {type(e).__name__})"
+        torch.cuda.synchronize()
     K = args.steps
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
     sampler = ClockSampler(smi_index(str(torch.cuda.get_device_properties(0).uuid), 0))
@@ -433,7 +447,7 @@ def run_other_workload(args):
     for i in range(K):
         flush.zero_()
         ev[i][0].record()
-        step()
+        run()
         ev[i][1].record()
     torch.cuda.synchronize()
     clocks = sampler.stop()
@@ -456,7 +470,7 @@ def run_other_workload(args):
     line = {"metric": f"{wl.name}: {unit}", "value": units * 1000.0 / ms, "unit": unit, "n_gpus": 1,
             "steps": K, "warmup": max(3, args.warmup), "ms_per_step": ms, "higher_is_better": True,
             "dtype": wl.dt, "data": "synthetic (seeded PCG64)",
-            "config": {"workload": wl.name, "step": what,
+            "config": {"workload": wl.name, "step": what, "issue": how,
                        "l2": "flushed before every timed step (256 MiB write); events bracket the step"},
             "algorithmic": {"bytes_per_step": byts, "flops_per_step": flops, "achieved_gbs": gbs,
                             "frac_of_measured_hbm": gbs / hbm, "achieved_tflops": tfs,
@@ -466,8 +480,61 @@ def run_other_workload(args):
             "clocks": clocks}
     if wid == 3:
         line["hca_compress"] = time_hca_compress(wl, csa, torch, flush, min(K, 20), hbm)
+    if wid == 5:
+        line["compress_step"] = time_compress_step(wl, csa, torch, D, flush, min(K, 20))
     print(json.dumps(line))
     return 0
+
+
+def time_compress_step(wl, csa, torch, D, flush, K):
+    """The decode-time compressors of the layer pair in their most expensive
+    step: every sequence's newest token completes both a CSA block (both
+    caches get an entry) and an HCA block (lengths rounded down to a
+    multiple of 128); tokens from the 128-token window ring."""
+    s = wl.sizes
+    B, d, dI, m = s["B"], s["d"], s["dI"], s["m"]
+    lens = to_dev_i32(torch, (wl["lens"] // m) * m)
+    g = lambda role, shape: torch.from_numpy(W.normal(9, role, shape, d ** -0.5, "bf16").view(np.int16)) \
+        .cuda().view(torch.bfloat16)
+    Wa, Wb, b8 = g("Wa", (d, d)), g("Wb", (d, d)), g("beta", (8, d))
+    kWa, kWb, kb8 = g("kWa", (dI, dI)), g("kWb", (dI, dI)), g("kbeta", (8, dI))
+    hW, hb = g("hca_W", (d, d)), g("hca_beta", (m, d))
+    ring = D["win"]
+    kv = torch.empty(B, s["nc"], d, dtype=torch.bfloat16, device="cuda")
+    kI = torch.empty(B, s["nc"], dI, dtype=torch.bfloat16, device="cuda")
+    hkv = torch.empty(B, s["hnc"], d, dtype=torch.bfloat16, device="cuda")
+
+    def step():
+        csa.csa_compress_step(ring, lens, Wa, Wb, b8, kv)
+        csa.csa_compress_step(ring, lens, kWa, kWb, kb8, kI)
+        csa.hca_compress_step(ring, lens, hW, hb, hkv, m=m)
+
+    for _ in range(3):
+        step()
+    # device time of the three kernels (the library's per-launch events): the
+    # host needs longer to issue three small calls than the GPU to run them
+    per = []
+    csa.set_kernel_timing(True)
+    for i in range(K):
+        flush.zero_()
+        tot = 0.0
+        for fn in (lambda: csa.csa_compress_step(ring, lens, Wa, Wb, b8, kv),
+                   lambda: csa.csa_compress_step(ring, lens, kWa, kWb, kb8, kI),
+                   lambda: csa.hca_compress_step(ring, lens, hW, hb, hkv, m=m)):
+            fn()
+            tot += sum(csa.kernel_timing())
+        per.append(tot)
+    csa.set_kernel_timing(False)
+    torch.cuda.synchronize()
+    csa.check_device_error()
+    return {"us": 1000 * statistics.median(per), "sequences": B,
+            "calls": "csa_compress_step (KV) + csa_compress_step (indexer keys) + hca_compress_step",
+            "timing": "sum of the three kernels' device times",
+            "note": "every sequence completes a CSA and an HCA block in this step"}
+
+
+def to_dev_i32(torch, a):
+    return torch.from_numpy(np.ascontiguousarray(a, dtype=np.int32)).cuda()
 
 
 def time_hca_compress(wl, csa, torch, flush, K, hbm):

@@ -9,6 +9,7 @@ built, or a tensor is not a contiguous CUDA tensor, the call raises.
 Entry points (method definitions are stated in ``include/csa.h``):
   csa_compress    CSA overlapping compressor (stride 4, 8-token windows)
   hca_compress    HCA compressor (stride m, no overlap)
+  csa_compress_step / hca_compress_step  the entry a decode token completes
   csa_index_topk  lightning-indexer scores + per-query top-k
   csa_index_topk_noalloc  the same without a workspace (fixed device scratch)
   csa_attend      MQA attention over the selected entries + sliding window
@@ -56,6 +57,8 @@ def lib() -> ctypes.CDLL:
         L.csa_check_device_error.argtypes = [P]
         L.csa_compress.argtypes = [P, P, I, I, I, P, P, P, I, P, P]
         L.hca_compress.argtypes = [P, P, I, I, I, I, P, P, I, P, P]
+        L.csa_compress_step.argtypes = [P, I, P, I, I, P, P, P, I, P, I, P]
+        L.hca_compress_step.argtypes = [P, I, P, I, I, I, P, P, I, P, I, P]
         L.csa_index_topk_workspace_size.argtypes = [I, I, I, I]
         L.csa_index_topk_workspace_size.restype = S
         L.csa_index_topk.argtypes = [P, P, P, P, P, I, I, I, I, I, I, I, P, P, P, S, P]
@@ -64,9 +67,10 @@ def lib() -> ctypes.CDLL:
         L.csa_index_topk_noalloc_max_elems.restype = S
         L.csa_index_scores.argtypes = [P, P, P, P, P, I, I, I, I, I, I, P, P]
         L.csa_topk.argtypes = [P, P, P, I, I, I, I, P, P]
-        L.csa_attend.argtypes = [P, P, P, I, P, P, P, I, I, I, I, I, I, I, F, I, P, P]
-        L.hca_attend.argtypes = [P, P, P, I, P, P, I, I, I, I, I, I, I, F, I, P, P]
-        for name in ("csa_check_device_error", "csa_compress", "hca_compress", "csa_index_topk",
+        L.csa_attend.argtypes = [P, P, P, I, P, P, P, I, I, I, I, I, I, I, F, P, I, P, P]
+        L.hca_attend.argtypes = [P, P, P, I, P, P, I, I, I, I, I, I, I, F, P, I, P, P]
+        for name in ("csa_check_device_error", "csa_compress", "hca_compress", "csa_compress_step",
+                     "hca_compress_step", "csa_index_topk",
                      "csa_index_topk_noalloc", "csa_index_scores", "csa_topk", "csa_attend", "hca_attend"):
             getattr(L, name).restype = I
         _lib = L
@@ -138,6 +142,25 @@ def hca_compress(x, lens, W, bias, m=128, out=None, stream=None):
     _check(lib().hca_compress(_p(x), _i32(lens), B, n_max, d, m, _p(W), _p(bias), _dt(x), _p(out),
                               _s(stream)))
     return out
+
+
+def csa_compress_step(x_tok, lens, W_a, W_b, bias8, cache, stream=None):
+    """Decode-time CSA compressor: for every sequence whose newest token
+    completes a 4-token block, entry lens/4 - 1 of cache [B][nc_max][d] from
+    the token ring x_tok [B][n_tok][d] (token s at row s % n_tok)."""
+    B, n_tok, d = x_tok.shape
+    _check(lib().csa_compress_step(_p(x_tok), n_tok, _i32(lens), B, d, _p(W_a), _p(W_b), _p(bias8),
+                                   _dt(x_tok), _p(cache), cache.shape[1], _s(stream)))
+    return cache
+
+
+def hca_compress_step(x_tok, lens, W, bias, cache, m=128, stream=None):
+    """Decode-time HCA compressor: entry lens/m - 1 of cache for every
+    sequence whose newest token completes an m-token block."""
+    B, n_tok, d = x_tok.shape
+    _check(lib().hca_compress_step(_p(x_tok), n_tok, _i32(lens), B, d, m, _p(W), _p(bias), _dt(x_tok),
+                                   _p(cache), cache.shape[1], _s(stream)))
+    return cache
 
 
 def index_topk_workspace_size(B, Tq, nc_max, has_scores_out=False) -> int:
@@ -230,27 +253,34 @@ def csa_topk(scores, lens, k, q_pos=None, idx_out=None, stream=None):
     return idx_out
 
 
+def _f32(t):
+    """Device pointer of a contiguous float32 CUDA tensor (None -> NULL)."""
+    if t is not None and t.dtype != torch.float32:
+        raise TypeError("expected a float32 tensor")
+    return _p(t)
+
+
 def csa_attend(q, kv_c, kv_tok, idx, lens, q_pos=None, window=128, scale=0.0, out=None,
-               stream=None):
+               stream=None, sink=None):
     """q [B][Tq][H][d], kv_c [B][nc_max][d], kv_tok [B][n_tok][d] (ring),
-    idx [B][Tq][k] -> out [B][Tq][H][d]."""
+    idx [B][Tq][k], sink [H] float32 or None -> out [B][Tq][H][d]."""
     B, Tq, H, d = q.shape
     if out is None:
         out = torch.empty_like(q)
     _check(lib().csa_attend(_p(q), _p(kv_c), _p(kv_tok), kv_tok.shape[1], _i32(idx), _i32(lens),
                             _i32(q_pos), B, Tq, H, d, kv_c.shape[1], idx.shape[-1], window,
-                            float(scale), _dt(q), _p(out), _s(stream)))
+                            float(scale), _f32(sink), _dt(q), _p(out), _s(stream)))
     return out
 
 
 def hca_attend(q, kv_c, kv_tok, lens, q_pos=None, m=128, window=128, scale=0.0, out=None,
-               stream=None):
-    """q [B][Tq][H][d], kv_c [B][nc_max][d], kv_tok [B][n_tok][d] (ring)
-    -> out [B][Tq][H][d]."""
+               stream=None, sink=None):
+    """q [B][Tq][H][d], kv_c [B][nc_max][d], kv_tok [B][n_tok][d] (ring),
+    sink [H] float32 or None -> out [B][Tq][H][d]."""
     B, Tq, H, d = q.shape
     if out is None:
         out = torch.empty_like(q)
     _check(lib().hca_attend(_p(q), _p(kv_c), _p(kv_tok), kv_tok.shape[1], _i32(lens), _i32(q_pos),
-                            B, Tq, H, d, kv_c.shape[1], m, window, float(scale), _dt(q), _p(out),
-                            _s(stream)))
+                            B, Tq, H, d, kv_c.shape[1], m, window, float(scale), _f32(sink), _dt(q),
+                            _p(out), _s(stream)))
     return out

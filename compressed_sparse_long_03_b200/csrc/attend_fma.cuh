@@ -42,9 +42,17 @@ struct AttendArgs {
   const int32_t *lens;
   const int32_t *q_pos;
   void *out;
+  const float *sink;  // [H] per-head sink logits (scaled-logit units), or nullptr
   int n_tok, k, Tq, H, nc_max, m, window;
   float scale_log2;  // softmax scale * log2(e)
 };
+
+// A head's sink logit in the kernels' base-2 units (-inf: no sink).  "Anatomy
+// of a Frontier Model", second of the three details: a learned per-head logit
+// whose exponential joins the softmax denominator (it carries no value).
+__device__ __forceinline__ float sink_log2(const AttendArgs &a, int h) {
+  return a.sink ? __ldg(a.sink + h) * 1.4426950408889634f : -INFINITY;
+}
 
 template <int CS>
 __device__ __forceinline__ void att_cluster_sync() {
@@ -204,10 +212,11 @@ __global__ void __launch_bounds__(kAttThreads) k_attend_fma(AttendArgs a) {
   const int nmine = (H - rank + CS - 1) / CS;
   for (int u = tid; u < nmine * D; u += kAttThreads) {
     const int h = rank + CS * (u / D), e = u % D;
-    float M = -INFINITY;
+    const float sk = sink_log2(a, h);
+    float M = sk;
 #pragma unroll
     for (int c = 0; c < CS; ++c) M = fmaxf(M, att_peer<CS>(pm, c)[h]);
-    float Ls = 0.f, Os = 0.f;
+    float Ls = sk == -INFINITY ? 0.f : exp2f(sk - M), Os = 0.f;
 #pragma unroll
     for (int c = 0; c < CS; ++c) {
       const float mc = att_peer<CS>(pm, c)[h];

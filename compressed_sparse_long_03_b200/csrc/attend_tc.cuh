@@ -320,10 +320,11 @@ __global__ void __launch_bounds__(kAtThreads, 1) k_attend_tc(AttendArgs a) {
   // merge weights of this CTA's heads (h = rank + CS * hl), ranks in order
   const int nmine = (H - rank + CS - 1) / CS;
   if (tid < nmine) {
-    float M = -INFINITY;
+    const float sk = sink_log2(a, rank + CS * tid);
+    float M = sk;
 #pragma unroll
     for (int c = 0; c < CS; ++c) M = fmaxf(M, pm[tid * CS + c]);
-    float Ls = 0.f;
+    float Ls = sk == -INFINITY ? 0.f : ex2(sk - M);
 #pragma unroll
     for (int c = 0; c < CS; ++c) {
       const float mc = pm[tid * CS + c];

@@ -8,9 +8,9 @@
 // overlap.  "The Exchange Rates of a Million Tokens", section 3: the two
 // overlapping series share one joint softmax.
 //
-// Both kernels run on the CUDA cores: the logit contraction is d x d per
-// token (0.5 GFLOP for a whole 8K-token prefill), small next to the rest of
-// the path; the pooling itself is per channel.
+// These CUDA-core kernels serve fp32 and d = 32 (bf16 with d in {64, 128}
+// runs on the tensor cores, compress_tc.cuh); the pooling itself is per
+// channel.
 #pragma once
 
 #include "common.cuh"
@@ -48,6 +48,7 @@ __global__ void __launch_bounds__(D) k_csa_compress(const T *__restrict__ x,
   const long s0 = 4L * (i0 - 1);  // token of xs[0]
 
   // stage the tokens (fp32) in shared memory, zero outside the sequence
+#pragma unroll
   for (int u = 0; u < NTOK; ++u) {
     const long s = s0 + u;
     float v = 0.f;
@@ -61,13 +62,22 @@ __global__ void __launch_bounds__(D) k_csa_compress(const T *__restrict__ x,
   float za[4 * E], zb[4 * E];
 #pragma unroll
   for (int u = 0; u < 4 * E; ++u) za[u] = zb[u] = 0.f;
-  for (int e = 0; e < D; ++e) {
-    const float wa = to_f(Wa[(size_t)e * D + c]);
-    const float wb = to_f(Wb[(size_t)e * D + c]);
+  // this thread's weight column, 16 inputs at a time with all loads in
+  // flight (one round trip per block instead of one per input)
+  for (int e0 = 0; e0 < D; e0 += 16) {
+    float wa[16], wb[16];
 #pragma unroll
-    for (int u = 0; u < 4 * E; ++u) {
-      za[u] = fmaf(xs[u][e], wa, za[u]);
-      zb[u] = fmaf(xs[u + 4][e], wb, zb[u]);
+    for (int ee = 0; ee < 16; ++ee) {
+      wa[ee] = to_f(Wa[(size_t)(e0 + ee) * D + c]);
+      wb[ee] = to_f(Wb[(size_t)(e0 + ee) * D + c]);
+    }
+#pragma unroll
+    for (int ee = 0; ee < 16; ++ee) {
+#pragma unroll
+      for (int u = 0; u < 4 * E; ++u) {
+        za[u] = fmaf(xs[u][e0 + ee], wa[ee], za[u]);
+        zb[u] = fmaf(xs[u + 4][e0 + ee], wb[ee], zb[u]);
+      }
     }
   }
   float bias[8];
@@ -135,16 +145,22 @@ __global__ void __launch_bounds__(D) k_hca_compress(const T *__restrict__ x,
     for (long j0 = 0; j0 < cnt; j0 += kHcaChunk) {
       const int len = (int)((cnt - j0) < kHcaChunk ? (cnt - j0) : kHcaChunk);
       __syncthreads();
+#pragma unroll
       for (int u = 0; u < kHcaChunk; ++u)
         xs[u][c] = (u < len) ? to_f(x[((size_t)b * n_max + first + j0 + u) * D + c]) : 0.f;
       __syncthreads();
       float z[kHcaChunk];
 #pragma unroll
       for (int u = 0; u < kHcaChunk; ++u) z[u] = 0.f;
-      for (int e = 0; e < D; ++e) {
-        const float we = to_f(W[(size_t)e * D + c]);
+      for (int e0 = 0; e0 < D; e0 += 16) {
+        float we[16];
 #pragma unroll
-        for (int u = 0; u < kHcaChunk; ++u) z[u] = fmaf(xs[u][e], we, z[u]);
+        for (int ee = 0; ee < 16; ++ee) we[ee] = to_f(W[(size_t)(e0 + ee) * D + c]);
+#pragma unroll
+        for (int ee = 0; ee < 16; ++ee) {
+#pragma unroll
+          for (int u = 0; u < kHcaChunk; ++u) z[u] = fmaf(xs[u][e0 + ee], we[ee], z[u]);
+        }
       }
       float cmax = -INFINITY;
 #pragma unroll

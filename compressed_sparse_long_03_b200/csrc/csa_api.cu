@@ -22,6 +22,7 @@
 #include "common.cuh"
 #include "compress.cuh"
 #include "compress_tc.cuh"
+#include "compress_step.cuh"
 #include "index_score_fma.cuh"
 #include "index_score_tc.cuh"
 #include "topk.cuh"
@@ -262,6 +263,33 @@ int launch_compress_tc(const void *x, const int32_t *lens, int B, int n_max, int
   return launch_cluster(kern, 1, grid, csa::kCtThreads, smem, st, what, tmX, a);
 }
 
+// decode-time compressors: grid = sequences, block = channels
+template <typename T, int D>
+int launch_compress_step(bool is_csa, const void *tok, int n_tok, const int32_t *lens, int B, int m,
+                         const void *Wa, const void *Wb, const void *bias, void *cache, int nc_max,
+                         cudaStream_t st, const char *what) {
+  auto X = static_cast<const T *>(tok);
+  auto A = static_cast<const T *>(Wa);
+  auto Z = static_cast<const T *>(bias);
+  auto O = static_cast<T *>(cache);
+  if (is_csa)
+    return launch_cluster(csa::k_csa_compress_step<T, D>, 1, (unsigned)B, D, 0, st, what, X, n_tok,
+                          lens, A, static_cast<const T *>(Wb), Z, O, nc_max);
+  return launch_cluster(csa::k_hca_compress_step<T, D>, csa::kStepCluster, (unsigned)B * csa::kStepCluster,
+                        D, 0, st, what, X, n_tok, lens, m, A, Z, O, nc_max);
+}
+
+template <typename T>
+int compress_step_d(bool is_csa, const void *tok, int n_tok, const int32_t *lens, int B, int d, int m,
+                    const void *Wa, const void *Wb, const void *bias, void *cache, int nc_max,
+                    cudaStream_t st, const char *what) {
+  switch (d) {
+    case 32: return launch_compress_step<T, 32>(is_csa, tok, n_tok, lens, B, m, Wa, Wb, bias, cache, nc_max, st, what);
+    case 64: return launch_compress_step<T, 64>(is_csa, tok, n_tok, lens, B, m, Wa, Wb, bias, cache, nc_max, st, what);
+    default: return launch_compress_step<T, 128>(is_csa, tok, n_tok, lens, B, m, Wa, Wb, bias, cache, nc_max, st, what);
+  }
+}
+
 template <typename T>
 int launch_csa_compress(const void *x, const int32_t *lens, int B, int n_max, int d, const void *Wa,
                         const void *Wb, const void *b8, void *out, cudaStream_t st) {
@@ -462,8 +490,8 @@ int launch_attend_tc(const csa::AttendArgs &a, int R, cudaStream_t st, const cha
 
 int attend_common(const void *q, const void *kv_c, const void *kv_tok, int n_tok,
                   const int32_t *idx, const int32_t *lens, const int32_t *q_pos, int B, int Tq,
-                  int H, int d, int nc_max, int k, int m, int window, float scale, csa_dtype dt,
-                  void *out, void *stream, const char *what) {
+                  int H, int d, int nc_max, int k, int m, int window, float scale,
+                  const float *sink, csa_dtype dt, void *out, void *stream, const char *what) {
   int rc = check_dtype(dt, what);
   if (rc) return rc;
   if (B < 0 || Tq < 0) return fail(CSA_ERR_SHAPE, "%s: B=%d and Tq=%d must be >= 0", what, B, Tq);
@@ -487,6 +515,7 @@ int attend_common(const void *q, const void *kv_c, const void *kv_tok, int n_tok
   a.lens = lens;
   a.q_pos = q_pos;
   a.out = out;
+  a.sink = sink;
   a.n_tok = n_tok;
   a.k = k;
   a.Tq = Tq;
@@ -583,6 +612,41 @@ int hca_compress(const void *x, const int32_t *lens, int B, int n_max, int d, in
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (dt == CSA_F32) return launch_hca_compress<float>(x, lens, B, n_max, d, m, W, bias, out, st);
   return launch_hca_compress<__nv_bfloat16>(x, lens, B, n_max, d, m, W, bias, out, st);
+}
+
+static int compress_step_common(bool is_csa, const void *tok, int n_tok, const int32_t *lens, int B,
+                                int d, int m, const void *Wa, const void *Wb, const void *bias,
+                                csa_dtype dt, void *cache, int nc_max, void *stream,
+                                const char *what) {
+  begin_call();
+  int rc = check_dtype(dt, what);
+  if (rc) return rc;
+  if (d != 32 && d != 64 && d != 128) return fail(CSA_ERR_UNSUPPORTED, "%s: d=%d not in {32,64,128}", what, d);
+  if (!is_csa && (m < 1 || m > 4096)) return fail(CSA_ERR_UNSUPPORTED, "%s: m=%d not in [1,4096]", what, m);
+  if (B < 0 || n_tok < 1 || nc_max < 0)
+    return fail(CSA_ERR_SHAPE, "%s: B >= 0, n_tok >= 1, nc_max >= 0 required", what);
+  if (B == 0 || nc_max == 0) return CSA_OK;
+  if (!tok || !lens || !Wa || (is_csa && !Wb) || !bias || !cache)
+    return fail(CSA_ERR_NULL, "%s: a required pointer is NULL", what);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (dt == CSA_F32)
+    return compress_step_d<float>(is_csa, tok, n_tok, lens, B, d, m, Wa, Wb, bias, cache, nc_max, st, what);
+  return compress_step_d<__nv_bfloat16>(is_csa, tok, n_tok, lens, B, d, m, Wa, Wb, bias, cache, nc_max, st,
+                                        what);
+}
+
+int csa_compress_step(const void *x_tok, int n_tok, const int32_t *lens, int B, int d, const void *W_a,
+                      const void *W_b, const void *bias8, csa_dtype dt, void *cache, int nc_max,
+                      void *stream) {
+  return compress_step_common(true, x_tok, n_tok, lens, B, d, 4, W_a, W_b, bias8, dt, cache, nc_max,
+                              stream, "csa_compress_step");
+}
+
+int hca_compress_step(const void *x_tok, int n_tok, const int32_t *lens, int B, int d, int m,
+                      const void *W, const void *bias, csa_dtype dt, void *cache, int nc_max,
+                      void *stream) {
+  return compress_step_common(false, x_tok, n_tok, lens, B, d, m, W, nullptr, bias, dt, cache, nc_max,
+                              stream, "hca_compress_step");
 }
 
 size_t csa_index_topk_workspace_size(int B, int Tq, int nc_max, int has_scores_out) {
@@ -725,22 +789,24 @@ int csa_index_topk(const void *q_idx, const void *w, const void *k_idx, const in
 
 int csa_attend(const void *q, const void *kv_c, const void *kv_tok, int n_tok, const int32_t *idx,
                const int32_t *lens, const int32_t *q_pos, int B, int Tq, int H, int d, int nc_max,
-               int k, int window, float scale, csa_dtype dt, void *out, void *stream) {
+               int k, int window, float scale, const float *sink, csa_dtype dt, void *out,
+               void *stream) {
   begin_call();
   if (k < 1 || k > 4096) return fail(CSA_ERR_UNSUPPORTED, "csa_attend: k=%d not in [1,4096]", k);
   if (!idx && (long)B * Tq > 0) return fail(CSA_ERR_NULL, "csa_attend: idx is NULL");
   return attend_common(q, kv_c, kv_tok, n_tok, idx, lens, q_pos, B, Tq, H, d, nc_max, k, 4, window,
-                       scale, dt, out, stream, "csa_attend");
+                       scale, sink, dt, out, stream, "csa_attend");
 }
 
 int hca_attend(const void *q, const void *kv_c, const void *kv_tok, int n_tok,
                const int32_t *lens, const int32_t *q_pos, int B, int Tq, int H, int d, int nc_max,
-               int m, int window, float scale, csa_dtype dt, void *out, void *stream) {
+               int m, int window, float scale, const float *sink, csa_dtype dt, void *out,
+               void *stream) {
   begin_call();
   if (m < 1 || m > 4096) return fail(CSA_ERR_UNSUPPORTED, "hca_attend: m=%d not in [1,4096]", m);
   if (nc_max > 65536) return fail(CSA_ERR_UNSUPPORTED, "hca_attend: nc_max=%d > 65536", nc_max);
   return attend_common(q, kv_c, kv_tok, n_tok, nullptr, lens, q_pos, B, Tq, H, d, nc_max, 0, m,
-                       window, scale, dt, out, stream, "hca_attend");
+                       window, scale, sink, dt, out, stream, "hca_attend");
 }
 
 }  // extern "C"

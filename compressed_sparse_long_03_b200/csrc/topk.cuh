@@ -81,6 +81,18 @@ __device__ __forceinline__ void cluster_barrier() {
   }
 }
 
+// The cluster barrier split in two: arrive once this CTA has finished
+// reading its peers' shared memory, wait before leaving (so that no CTA
+// exits while a peer may still read it).
+template <int CS>
+__device__ __forceinline__ void cluster_arrive_release() {
+  if constexpr (CS > 1) asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+template <int CS>
+__device__ __forceinline__ void cluster_wait_acquire() {
+  if constexpr (CS > 1) asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
 template <int CS, typename P>
 __device__ __forceinline__ P *peer_ptr(P *mine, int rank) {
   if constexpr (CS > 1) {
@@ -197,9 +209,13 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(const float *__restrict__
         const int u = u0 + i * NT + tid;
         f[i] = u < nvec ? __ldg(vsrc + u) : make_float4(0.f, 0.f, 0.f, 0.f);
       }
+      // the lanes of a warp hold consecutive vectors; the 8 vectors of one
+      // 32-position group form a run of lanes (cut at the warp's edges)
+      const int r0 = (((head + p0) >> 2) + u0 + tid) & 7;  // this lane's place in its group
 #pragma unroll
       for (int i = 0; i < UNR; ++i) {
         const int u = u0 + i * NT + tid;
+        uint32_t gmax = 0;
         if (u < nvec) {
           const uint4 kv = make_uint4(order_key(f[i].x), order_key(f[i].y), order_key(f[i].z),
                                       order_key(f[i].w));
@@ -210,8 +226,13 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(const float *__restrict__
           atomicAdd(&sh.hist[b1], 1);
           atomicAdd(&sh.hist[b2], 1);
           atomicAdd(&sh.hist[b3], 1);
-          atomicMax(&gmaxbin[(head + 4 * u + p0) >> 5], (uint32_t)max(max(b0, b1), max(b2, b3)));
+          gmax = (uint32_t)max(max(b0, b1), max(b2, b3));
         }
+        // group maximum over the run (NT is a multiple of 8: r0 holds for every i)
+        const int lo_l = max(0, lane - r0), hi_l = min(31, lane + 7 - r0);
+        const unsigned seg = (hi_l == 31 ? 0xffffffffu : ((1u << (hi_l + 1)) - 1u)) & ~((1u << lo_l) - 1u);
+        gmax = __reduce_max_sync(seg, gmax);
+        if (lane == lo_l && u < nvec) atomicMax(&gmaxbin[(head + 4 * u + p0) >> 5], gmax);
       }
     }
     for (int j = head + 4 * nvec + tid; j < len; j += NT) take(j, __ldg(src + j));
@@ -225,27 +246,49 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(const float *__restrict__
     atomicAdd(&sh.super[(BPT * tid) / (kScoreBins / kTopkSuper)], sum);
   }
 
-  // ---- B: merge over the cluster: super-bins, then the bins of one
+  // ---- B: merge over the cluster, in warp 0: the 64 super-bins summed over
+  // the CTAs (two per lane, all loads in flight), the super-bin holding the
+  // k-th largest key by a warp scan from the top, then its 64 bins likewise
   cluster_barrier<CS>();  // [1]
-  {
-    int c1 = 0;
-    if (tid < kTopkSuper) {
+  static_assert(kTopkSuper == 64 && kScoreBins / kTopkSuper == 64, "two buckets per lane");
+  if (wid == 0) {
+    // descending: lane l holds buckets 63-2l (hi) and 62-2l (lo) of `arr`;
+    // returns {bucket, count above it, count in it} for the need-th key
+    auto pick = [&](const int *arr_mine, int need, int &bucket, int &above, int &cnt) {
+      int ch = 0, cl = 0;
 #pragma unroll
-      for (int c = 0; c < CS; ++c) c1 += peer_ptr<CS>(&sh, c)->super[kTopkSuper - 1 - tid];
-    }
-    find_bucket(sh, kTopkSuper, k, c1);
-    const int sstar = sh.info[0], above_s = sh.info[1];
-    __syncthreads();  // info is rewritten below
-    constexpr int Wb = kScoreBins / kTopkSuper;
-    int c2 = 0;
-    if (tid < Wb) {
+      for (int c = 0; c < CS; ++c) {
+        const int *arr = peer_ptr<CS>(arr_mine, c);
+        ch += arr[63 - 2 * lane];
+        cl += arr[62 - 2 * lane];
+      }
+      int incl = ch + cl;
 #pragma unroll
-      for (int c = 0; c < CS; ++c) c2 += peer_ptr<CS>(&sh, c)->hist[Wb * sstar + Wb - 1 - tid];
-    }
-    find_bucket(sh, Wb, k - above_s, c2);
-    if (tid == 0) {
-      sh.info[0] += Wb * sstar;
-      sh.info[1] += above_s;
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      const unsigned hit = __ballot_sync(0xffffffffu, incl >= need);
+      const int f = __ffs(hit) - 1;  // hit != 0: the row holds more than k keys
+      const int ex = __shfl_sync(0xffffffffu, incl - ch - cl, f);
+      const int fch = __shfl_sync(0xffffffffu, ch, f), fcl = __shfl_sync(0xffffffffu, cl, f);
+      if (ex + fch >= need) {
+        bucket = 63 - 2 * f;
+        above = ex;
+        cnt = fch;
+      } else {
+        bucket = 62 - 2 * f;
+        above = ex + fch;
+        cnt = fcl;
+      }
+    };
+    int sstar, above_s, cnt_s, bin, above_b, cnt_b;
+    pick(sh.super, k, sstar, above_s, cnt_s);
+    pick(sh.hist + 64 * sstar, k - above_s, bin, above_b, cnt_b);
+    if (lane == 0) {
+      sh.info[0] = 64 * sstar + bin;
+      sh.info[1] = above_s + above_b;
+      sh.info[2] = cnt_b;
     }
   }
   __syncthreads();
@@ -308,6 +351,10 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(const float *__restrict__
         sh.all_idx[m] = min(v, c * per) + peer_ptr<CS>(cand_pos, c)[u];
         sh.all_cta[m] = (unsigned char)c;
       }
+    }
+    // no more reads of peers' shared memory by this CTA: [3] arrive
+    cluster_arrive_release<CS>();
+    if (mode == 1) {
       for (int j = tid; j < 256; j += NT) sh.hist[j] = 0;
       __syncthreads();
       // radix step on bits 19..12 of the candidates (all share bits 31..20)
@@ -379,7 +426,7 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(const float *__restrict__
       }
       pos += __popc(mall);
     }
-    cluster_barrier<CS>();  // [3] peers may still read this CTA's shared memory
+    cluster_wait_acquire<CS>();  // [3] wait: peers may still read this CTA's shared memory
     return;
   }
 

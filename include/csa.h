@@ -135,6 +135,36 @@ CSA_API int hca_compress(const void *x, const int32_t *lens, int B, int n_max, i
                  const void *W, const void *bias, csa_dtype dt, void *out, void *stream);
 
 /* ------------------------------------------------------------------------
+ * csa_compress_step / hca_compress_step -- the compressors at decode: the
+ * one entry that the newest token completes.
+ *
+ * Anatomy page, "The attention: compress, then select", first of the three
+ * details: an entry is formed only once its block is complete (until then
+ * its tokens are reached through the sliding window).  For each sequence b
+ * with lens[b] > 0 and lens[b] a multiple of the stride (4, or m), the entry
+ * i = lens[b]/stride - 1 is computed exactly as csa_compress / hca_compress
+ * compute it (CSA: tokens 4i-4 .. 4i+3, entry 0 masked to its own block;
+ * HCA: tokens m*i .. m*i+m-1) and written to cache[b][i]; every other row
+ * and every other sequence is left untouched.  The tokens are read from the
+ * ring the decode step keeps for the window: token s at row s % n_tok of
+ * x_tok[b], which must hold the entry's tokens (n_tok >= min(8, lens[b])
+ * for CSA, >= m for HCA; otherwise the device error word is set).
+ *
+ *   x_tok  [B][n_tok][d]   token ring (key-value vectors or indexer keys)
+ *   lens   [B]             tokens of each sequence, newest included
+ *   W_a, W_b, bias8 / W, bias   as for csa_compress / hca_compress
+ *   cache  [B][nc_max][d]  the compressed cache, updated in place
+ * Supported: d in {32, 64, 128}; 1 <= m <= 4096.
+ * ---------------------------------------------------------------------- */
+CSA_API int csa_compress_step(const void *x_tok, int n_tok, const int32_t *lens, int B, int d,
+                              const void *W_a, const void *W_b, const void *bias8, csa_dtype dt,
+                              void *cache, int nc_max, void *stream);
+
+CSA_API int hca_compress_step(const void *x_tok, int n_tok, const int32_t *lens, int B, int d, int m,
+                              const void *W, const void *bias, csa_dtype dt, void *cache, int nc_max,
+                              void *stream);
+
+/* ------------------------------------------------------------------------
  * csa_index_topk -- lightning-indexer scores and per-query top-k.
  *
  * Anatomy page, CSA bullet: a small lightning indexer (64 heads of 128
@@ -236,13 +266,18 @@ CSA_API int csa_index_topk_noalloc(const void *q_idx, const void *w, const void 
  *                             (min(window, t+1) <= n_tok)
  *   idx    [B][Tq][k] int32   selected entries (csa_index_topk output)
  *   scale  softmax scale; <= 0 means 1/sqrt(d)
+ *   sink   [H] float or NULL: per-head sink logit s_h (second of the three
+ *          details: a learned logit whose exponential joins the softmax
+ *          denominator; it carries no value), in the units of the scaled
+ *          logits: o = sum_j e^{l_j} v_j / (sum_j e^{l_j} + e^{s_h})
  *   out    [B][Tq][H][d]
  * Supported: d in {64, 128}; 1 <= H <= 128; 1 <= k <= 4096;
  * 1 <= window <= 4096.
  * ---------------------------------------------------------------------- */
 CSA_API int csa_attend(const void *q, const void *kv_c, const void *kv_tok, int n_tok, const int32_t *idx,
                const int32_t *lens, const int32_t *q_pos, int B, int Tq, int H, int d, int nc_max,
-               int k, int window, float scale, csa_dtype dt, void *out, void *stream);
+               int k, int window, float scale, const float *sink, csa_dtype dt, void *out,
+               void *stream);
 
 /* ------------------------------------------------------------------------
  * hca_attend -- dense MQA attention over every visible HCA entry + window.
@@ -256,7 +291,8 @@ CSA_API int csa_attend(const void *q, const void *kv_c, const void *kv_tok, int 
  * ---------------------------------------------------------------------- */
 CSA_API int hca_attend(const void *q, const void *kv_c, const void *kv_tok, int n_tok,
                const int32_t *lens, const int32_t *q_pos, int B, int Tq, int H, int d, int nc_max,
-               int m, int window, float scale, csa_dtype dt, void *out, void *stream);
+               int m, int window, float scale, const float *sink, csa_dtype dt, void *out,
+               void *stream);
 
 #ifdef __cplusplus
 }

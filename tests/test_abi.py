@@ -99,10 +99,10 @@ def att_call(L, fn="csa_attend", **kw):
     if fn == "csa_attend":
         return L.csa_attend(a["q"], a["kv"], a["tok"], a["n_tok"], a["idx"], a["lens"], a["q_pos"],
                             a["B"], a["Tq"], a["H"], a["d"], a["nc"], a["k"], a["window"],
-                            ctypes.c_float(a["scale"]), a["dt"], a["out"], None)
+                            ctypes.c_float(a["scale"]), None, a["dt"], a["out"], None)
     return L.hca_attend(a["q"], a["kv"], a["tok"], a["n_tok"], a["lens"], a["q_pos"], a["B"], a["Tq"],
                         a["H"], a["d"], a["nc"], a["m"], a["window"], ctypes.c_float(a["scale"]),
-                        a["dt"], a["out"], None)
+                        None, a["dt"], a["out"], None)
 
 
 def test_attend_validation(L):

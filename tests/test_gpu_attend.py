@@ -160,3 +160,39 @@ def test_invalid_window_ring_raises_device_error():
     with pytest.raises(csa.CsaError):
         csa.check_device_error()
     assert np.all(to_host(out) == 0)
+
+
+@pytest.mark.parametrize("dt,d,H,B,Tq,hca", [
+    ("bf16", 128, 64, 2, 1, False),   # tensor-core path, 8-CTA clusters
+    ("bf16", 128, 16, 2, 150, False),  # tensor-core path, one CTA per row
+    ("f32", 64, 8, 2, 3, False),      # CUDA-core path
+    ("bf16", 64, 12, 2, 2, False),    # CUDA-core path, bf16
+    ("bf16", 128, 64, 3, 1, True),    # HCA, tensor-core path
+])
+def test_attend_with_sink(dt, d, H, B, Tq, hca):
+    """Per-head sink logits (one far below every logit, one far above, the
+    rest moderate) on both attention kernels, against the oracle."""
+    torch = pytest.importorskip("torch")
+    seed = 300 + d + H + Tq
+    k, nc, window, n_tok = 256, 1500, 128, 6000
+    lens = np.array([4 * nc, 4 * nc - 9, 4 * nc - 100][:B], np.int32)
+    q = W.normal(seed, "q", (B, Tq, H, d), 1.0, dt)
+    kv = W.normal(seed, "kv", (B, nc, d), 1.0, dt)
+    tok = W.normal(seed, "win", (B, n_tok, d), 1.0, dt)
+    sink = (np.random.default_rng(seed).standard_normal(H) * 2.0).astype(np.float32)
+    sink[0] = -1e30
+    sink[-1] = 40.0
+    dsink = torch.from_numpy(sink).cuda()
+    if hca:
+        m = 4
+        out = csa.hca_attend(to_dev(q), to_dev(kv), to_dev(tok), to_dev(lens), m=m, window=window,
+                             sink=dsink)
+        ref = oracle.attend(q, kv, tok, lens, idx=None, m=m, window=window, sink=sink.astype(np.float64))
+    else:
+        vis = oracle.visible(lens, B, Tq, 4)
+        idx = random_idx(seed, B, Tq, k, vis, nc)
+        out = csa.csa_attend(to_dev(q), to_dev(kv), to_dev(tok), to_dev(idx), to_dev(lens),
+                             window=window, sink=dsink)
+        ref = oracle.attend(q, kv, tok, lens, idx=idx, window=window, sink=sink.astype(np.float64))
+    csa.check_device_error()
+    assert_close(to_host(out), ref, dt, "attend with sink")
