@@ -482,8 +482,68 @@ def run_other_workload(args):
         line["hca_compress"] = time_hca_compress(wl, csa, torch, flush, min(K, 20), hbm)
     if wid == 5:
         line["compress_step"] = time_compress_step(wl, csa, torch, D, flush, min(K, 20))
+    if not args.no_cpu_baseline:
+        line["cpu_baseline"] = oracle_sample(wid, wl)
     print(json.dumps(line))
     return 0
+
+
+def oracle_sample(wid, wl):
+    """The oracle (fp64 C, all host cores) on a bounded sample of the same
+    workload, in the line's unit."""
+    import oracle
+    cores = os.cpu_count() or 1
+    oracle.set_threads(cores)
+    s = wl.sizes
+    k, window = s.get("k"), s["window"]
+
+    def clock(fn):
+        t = time.perf_counter()
+        fn()
+        return time.perf_counter() - t
+
+    if wid in (1, 2):
+        rows = 1 if wid == 1 else 64
+        tc = clock(lambda: (oracle.csa_compress(wl["x"], wl["lens"], wl["Wa"], wl["Wb"], wl["beta"]),
+                            oracle.csa_compress(wl["kx"], wl["lens"], wl["kWa"], wl["kWb"], wl["kbeta"])))
+        C = oracle.round_to(oracle.csa_compress(wl["x"], wl["lens"], wl["Wa"], wl["Wb"], wl["beta"]),
+                            oracle.F32 if wl.dt == "f32" else oracle.BF16)
+        KI = oracle.round_to(oracle.csa_compress(wl["kx"], wl["lens"], wl["kWa"], wl["kWb"], wl["kbeta"]),
+                             oracle.F32 if wl.dt == "f32" else oracle.BF16)
+        n, Tq = s["n"], s["Tq"]
+        pos = np.linspace(n - Tq, n - 1, rows).astype(np.int32)[None, :]
+        sub = lambda a: a[:, pos[0] - (n - Tq)]
+
+        def rows_fn():
+            idx, _ = oracle.index_topk(sub(wl["qI"]), sub(wl["w"]), KI, wl["lens"], k, pos)
+            oracle.attend(sub(wl["q"]), C, wl["x"], wl["lens"], idx=idx, q_pos=pos, window=window)
+        tr = clock(rows_fn)
+        if wid == 1:
+            return {"value": 1.0 / (tc + tr), "unit": "queries/s", "cores": cores, "kind": "oracle",
+                    "sample": "one full decode step (both compressors, indexer + top-k, attention)"}
+        return {"value": Tq / (tc + tr * Tq / rows), "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                "sample": f"both compressors over the {n} tokens, then indexer + top-k + attention for "
+                          f"{rows} of the {Tq} query rows (spread over the sequence), scaled to all rows"}
+    if wid == 3:
+        nq = 4
+        sl = slice(0, nq)
+        t = clock(lambda: oracle.attend(wl["q"][sl], wl["hkv"][sl], wl["win"][sl], wl["lens"][sl], idx=None,
+                                        m=s["m"], window=window))
+        return {"value": nq / t, "unit": "queries/s", "cores": cores, "kind": "oracle",
+                "sample": f"HCA attention for {nq} of the {s['B']} sequences"}
+    if wid == 5:
+        nq = 2
+        sl = slice(0, nq)
+
+        def pair():
+            idx, _ = oracle.index_topk(wl["qI"][sl], wl["w"][sl], wl["kI"][sl], wl["lens"][sl], k)
+            oracle.attend(wl["q"][sl], wl["kv"][sl], wl["win"][sl], wl["lens"][sl], idx=idx, window=window)
+            oracle.attend(wl["q2"][sl], wl["hkv"][sl], wl["win"][sl], wl["lens"][sl], idx=None, m=s["m"],
+                          window=window)
+        t = clock(pair)
+        return {"value": nq / t, "unit": "queries/s", "cores": cores, "kind": "oracle",
+                "sample": f"the CSA + HCA step for {nq} of the {s['B']} sequences"}
+    raise KeyError(wid)
 
 
 def time_compress_step(wl, csa, torch, D, flush, K):
