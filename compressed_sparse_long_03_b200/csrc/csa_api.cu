@@ -360,10 +360,13 @@ int launch_index_fma(const void *qI, const void *w, const void *kI, const int32_
   return launch_status("csa_index_topk (scores)");
 }
 
-template <int N, int DI>
+// The tensor-core scoring kernel with G query rows per unit (N1 head slots
+// each; N1 * G <= 256).
+template <int N1, int G, int DI>
 int launch_index_tc(const void *qI, const void *w, const void *kI, const int32_t *lens,
                     const int32_t *q_pos, int R, int Tq, int HI, int nc_max, float *scores,
                     bool fill, cudaStream_t st) {
+  constexpr int N = N1 * G;
   const char *what = "csa_index_scores";
   CUtensorMap tmK, tmQ;
   const int B = R / Tq;
@@ -372,10 +375,10 @@ int launch_index_tc(const void *qI, const void *w, const void *kI, const int32_t
   rc = encode_bf16_2d(&tmQ, qI, DI, (uint64_t)R * HI, 64, N, what);
   if (rc) return rc;
   constexpr size_t A_STAGE = (size_t)csa::kTcRows * DI * 2, B_SLOT = (size_t)N * DI * 2;
-  const size_t budget = 227 * 1024 - 1024 - 2 * B_SLOT - 1024;  // align slack, barriers, statics
+  const size_t budget = 227 * 1024 - 1024 - 2 * B_SLOT - 1024 - (G > 1 ? 2 * N * 4 : 0);
   const int stages = (int)std::min<size_t>(5, budget / A_STAGE);
   const size_t smem = 1024 + stages * A_STAGE + 2 * B_SLOT + 8 * (2 * stages + 9);
-  auto kern = csa::k_index_score_tc<N, DI>;
+  auto kern = csa::k_index_score_tc<N1, G, DI>;
   rc = ensure_smem(kern, smem, what);
   if (rc) return rc;
   csa::IndexTcArgs a;
@@ -387,19 +390,35 @@ int launch_index_tc(const void *qI, const void *w, const void *kI, const int32_t
   a.HI = HI;
   a.nc_max = nc_max;
   a.R = R;
+  a.G = G;
+  a.gpb = (Tq + G - 1) / G;
+  a.U = B * a.gpb;
   a.stages = stages;
   a.fill_invisible = fill ? 1 : 0;
   return launch_cluster(kern, 1, (unsigned)num_sms(), csa::kTcThreads, smem, st, what, tmK, tmQ, a);
 }
 
+// Decode (one query row per sequence): one row per unit, the heads padded to
+// a power of two.  Several rows per sequence with HI a power of two from 16
+// to 128: units of G rows sharing each key tile (N = G HI = 256, or 64 for
+// HI = 16).
 template <int DI>
 int launch_index_tc_n(const void *qI, const void *w, const void *kI, const int32_t *lens,
                       const int32_t *q_pos, int R, int Tq, int HI, int nc_max, float *scores,
                       bool fill, cudaStream_t st) {
-  if (HI <= 16) return launch_index_tc<16, DI>(qI, w, kI, lens, q_pos, R, Tq, HI, nc_max, scores, fill, st);
-  if (HI <= 32) return launch_index_tc<32, DI>(qI, w, kI, lens, q_pos, R, Tq, HI, nc_max, scores, fill, st);
-  if (HI <= 64) return launch_index_tc<64, DI>(qI, w, kI, lens, q_pos, R, Tq, HI, nc_max, scores, fill, st);
-  return launch_index_tc<128, DI>(qI, w, kI, lens, q_pos, R, Tq, HI, nc_max, scores, fill, st);
+  if (Tq >= 2) {
+    switch (HI) {
+      case 16: return launch_index_tc<16, 4, DI>(qI, w, kI, lens, q_pos, R, Tq, HI, nc_max, scores, fill, st);
+      case 32: return launch_index_tc<32, 4, DI>(qI, w, kI, lens, q_pos, R, Tq, HI, nc_max, scores, fill, st);
+      case 64: return launch_index_tc<64, 4, DI>(qI, w, kI, lens, q_pos, R, Tq, HI, nc_max, scores, fill, st);
+      case 128: return launch_index_tc<128, 2, DI>(qI, w, kI, lens, q_pos, R, Tq, HI, nc_max, scores, fill, st);
+      default: break;
+    }
+  }
+  if (HI <= 16) return launch_index_tc<16, 1, DI>(qI, w, kI, lens, q_pos, R, Tq, HI, nc_max, scores, fill, st);
+  if (HI <= 32) return launch_index_tc<32, 1, DI>(qI, w, kI, lens, q_pos, R, Tq, HI, nc_max, scores, fill, st);
+  if (HI <= 64) return launch_index_tc<64, 1, DI>(qI, w, kI, lens, q_pos, R, Tq, HI, nc_max, scores, fill, st);
+  return launch_index_tc<128, 1, DI>(qI, w, kI, lens, q_pos, R, Tq, HI, nc_max, scores, fill, st);
 }
 
 template <int CS>

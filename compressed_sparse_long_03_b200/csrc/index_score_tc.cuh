@@ -22,10 +22,15 @@
 //   warps 2-5  epilogue: tcgen05.ld of the accumulator (warp w reads TMEM
 //           lanes 32*(w%4)..), score = sum_h w_h*max(d_h,0) in fp32, in a
 //           fixed head order, coalesced store of 128 scores
-// Work: the visible 128-entry tiles of all query rows, in row-major order,
-// cut into one contiguous range per CTA (so a CTA loads each query block
-// once); every role walks the same range.  Tiles past a row's visible
-// entries are never loaded.  All waits are time-bounded (sm100.cuh).
+// Work: the visible 128-entry tiles of all query units, in order, cut into
+// one contiguous range per CTA (so a CTA loads each query block once); every
+// role walks the same range.  A unit is one query row at decode; with
+// several query rows per sequence (prefill) it is G consecutive rows of one
+// sequence, whose G x HI query vectors form one B operand (N = G HI <= 256):
+// each key tile is then read once for G rows, and the epilogue produces G
+// scores per entry, each masked by its own row's visibility.  Tiles past a
+// unit's visible entries are never loaded.  All waits are time-bounded
+// (sm100.cuh).
 #pragma once
 
 #include "common.cuh"
@@ -42,6 +47,7 @@ struct IndexTcArgs {
   const int32_t *q_pos;
   float *scores;           // [R][nc_max]
   int Tq, HI, nc_max, R;
+  int G, gpb, U;           // rows per unit, units per sequence, units
   int stages;              // depth of the key-tile ring
   int fill_invisible;      // also write -inf past each row's visible entries
 };
@@ -62,24 +68,40 @@ __device__ __forceinline__ int tc_row_tiles(const IndexTcArgs &a, int r) {
   return (tc_row_visible(a, r) + kTcRows - 1) / kTcRows;
 }
 
-// Cursor over a contiguous range of the row-major list of visible tiles.
+// first query row and row count of unit u
+__device__ __forceinline__ int tc_unit_row0(const IndexTcArgs &a, int u) {
+  return (u / a.gpb) * a.Tq + (u % a.gpb) * a.G;
+}
+__device__ __forceinline__ int tc_unit_rows(const IndexTcArgs &a, int u) {
+  return min(a.G, a.Tq - (u % a.gpb) * a.G);
+}
+// tiles of unit u: the most any of its rows sees
+__device__ __forceinline__ int tc_unit_tiles(const IndexTcArgs &a, int u) {
+  const int r0 = tc_unit_row0(a, u), n = tc_unit_rows(a, u);
+  int t = 0;
+  for (int i = 0; i < n; ++i) t = max(t, tc_row_tiles(a, r0 + i));
+  return t;
+}
+
+// Cursor over a contiguous range of the unit-major list of visible tiles.
 struct TileWalk {
-  int r, j, tiles, left;
+  int r, j, tiles, left;  // r: the unit
   __device__ void advance(const IndexTcArgs &a) {
     if (--left <= 0) return;
     if (++j < tiles) return;
     j = 0;
     do {
       ++r;
-      tiles = tc_row_tiles(a, r);
-    } while (tiles == 0 && r + 1 < a.R);
+      tiles = tc_unit_tiles(a, r);
+    } while (tiles == 0 && r + 1 < a.U);
   }
 };
 
-template <int N, int DI>
+template <int N1, int G, int DI>
 __global__ void __launch_bounds__(kTcThreads, 1)
     k_index_score_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmQ,
                      IndexTcArgs a) {
+  constexpr int N = N1 * G;  // MMA N: G rows' query vectors (N1 heads each)
   using namespace sm100;
   constexpr int KATOMS = DI / 64;                       // 128-byte K slices
   constexpr uint32_t A_ATOM = kTcRows * 128;            // bytes per K slice of a key tile
@@ -94,6 +116,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   __shared__ int abort_flag;
   __shared__ int range[3];  // first row, first tile, tile count
   __shared__ int scan[33];
+  __shared__ float sw[2][G > 1 ? N : 1];  // grouped units: the G rows' head weights
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int S = a.stages;
@@ -134,10 +157,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
   // this CTA's contiguous share of the visible tiles
   {
-    const int per = (a.R + kTcThreads - 1) / kTcThreads;
-    const int rb = min(a.R, tid * per), re = min(a.R, rb + per);
+    const int per = (a.U + kTcThreads - 1) / kTcThreads;
+    const int rb = min(a.U, tid * per), re = min(a.U, rb + per);
     int mine = 0;
-    for (int r = rb; r < re; ++r) mine += tc_row_tiles(a, r);
+    for (int r = rb; r < re; ++r) mine += tc_unit_tiles(a, r);
     int total;
     const int before = block_exclusive_scan(mine, scan, &total);
     const long lo = (long)total * blockIdx.x / gridDim.x;
@@ -145,7 +168,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     if (lo < hi && before <= lo && lo < before + mine) {
       long acc = before;
       for (int r = rb; r < re; ++r) {
-        const int t = tc_row_tiles(a, r);
+        const int t = tc_unit_tiles(a, r);
         if (lo < acc + t) {
           range[0] = r;
           range[1] = (int)(lo - acc);
@@ -165,7 +188,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   wk.r = range[0];
   wk.j = range[1];
   wk.left = range[2];
-  wk.tiles = wk.left > 0 ? tc_row_tiles(a, wk.r) : 0;
+  wk.tiles = wk.left > 0 ? tc_unit_tiles(a, wk.r) : 0;
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -181,15 +204,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           mbar_arrive_expect_tx(q_full + 8 * slot, B_SLOT);
 #pragma unroll
           for (int ka = 0; ka < KATOMS; ++ka)
-            tma_load_2d(smem_u32(sB + slot * B_SLOT + ka * B_ATOM), &tmQ, 64 * ka, wk.r * a.HI,
-                        q_full + 8 * slot);
+            tma_load_2d(smem_u32(sB + slot * B_SLOT + ka * B_ATOM), &tmQ, 64 * ka,
+                        tc_unit_row0(a, wk.r) * a.HI, q_full + 8 * slot);
           ++nq;
           cur_r = wk.r;
         }
         const uint32_t s = nt % S;
         if (!(ok = mbar_wait(b_empty + 8 * s, ((nt / S) & 1) ^ 1, abort))) break;
         mbar_arrive_expect_tx(b_full + 8 * s, A_STAGE);
-        const int y = (wk.r / a.Tq) * a.nc_max + wk.j * kTcRows;
+        const int y = (wk.r / a.gpb) * a.nc_max + wk.j * kTcRows;
 #pragma unroll
         for (int ka = 0; ka < KATOMS; ++ka)
           tma_load_2d_hint(smem_u32(sA + s * A_STAGE + ka * A_ATOM), &tmK, 64 * ka, y, b_full + 8 * s,
@@ -244,16 +267,31 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     // ------------------------------------------------------------ epilogue
     const int quad = warp & 3;  // TMEM lanes 32*quad .. 32*quad+31
     const int row = quad * 32 + lane;
-    float wv[N];
-    int cur_r = -1, vis = 0;
+    float wv[G == 1 ? N1 : 1];
+    int vis[G];
+    int cur_u = -1, r0 = 0, nrows = 1, upar = 0;
     uint32_t nt = 0;
     for (; wk.left > 0; wk.advance(a)) {
-      if (wk.r != cur_r) {
-        cur_r = wk.r;
-        vis = tc_row_visible(a, cur_r);
+      if (wk.r != cur_u) {
+        cur_u = wk.r;
+        r0 = tc_unit_row0(a, cur_u);
+        nrows = tc_unit_rows(a, cur_u);
 #pragma unroll
-        for (int h = 0; h < N; ++h)
-          wv[h] = h < a.HI ? __bfloat162float(a.w[(size_t)cur_r * a.HI + h]) : 0.f;
+        for (int g = 0; g < G; ++g) vis[g] = g < nrows ? tc_row_visible(a, r0 + g) : 0;
+        if constexpr (G == 1) {
+#pragma unroll
+          for (int h = 0; h < N1; ++h)
+            wv[h] = h < a.HI ? __bfloat162float(a.w[(size_t)r0 * a.HI + h]) : 0.f;
+        } else {
+          // the unit's head weights into shared memory (the 4 epilogue warps;
+          // two buffers, so the previous unit's may still be read)
+          upar ^= 1;
+          for (int u = tid - 64; u < N; u += 128) {
+            const int g = u / N1, h = u % N1;
+            sw[upar][u] = (g < nrows && h < a.HI) ? __bfloat162float(a.w[(size_t)(r0 + g) * a.HI + h]) : 0.f;
+          }
+          asm volatile("bar.sync 1, 128;" ::: "memory");
+        }
       }
       const uint32_t acc = nt & 1;
       // every lane waits; the warp leaves together if any lane timed out, so
@@ -261,20 +299,40 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       const bool ok = mbar_wait(t_full + 8 * acc, (nt >> 1) & 1, abort);
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
-      uint32_t d[N];
       const uint32_t taddr = tmem + ((uint32_t)(quad * 32) << 16) + acc * N;
-#pragma unroll
-      for (int c = 0; c < N / 16; ++c) tmem_ld16(taddr + 16 * c, d + 16 * c);
-      tmem_wait_ld_regs<N>(d);
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(t_empty + 8 * acc);
-      float sc = 0.f;
-#pragma unroll
-      for (int h = 0; h < N; ++h) sc = fmaf(wv[h], fmaxf(__uint_as_float(d[h]), 0.f), sc);
       const int i = wk.j * kTcRows + row;
-      if (i < a.nc_max) a.scores[(size_t)cur_r * a.nc_max + i] = i < vis ? sc : -INFINITY;
-
+      if constexpr (G == 1) {
+        uint32_t d[N1];
+#pragma unroll
+        for (int c = 0; c < N1 / 16; ++c) tmem_ld16(taddr + 16 * c, d + 16 * c);
+        tmem_wait_ld_regs<N1>(d);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(t_empty + 8 * acc);
+        float sc = 0.f;
+#pragma unroll
+        for (int h = 0; h < N1; ++h) sc = fmaf(wv[h], fmaxf(__uint_as_float(d[h]), 0.f), sc);
+        if (i < a.nc_max) a.scores[(size_t)r0 * a.nc_max + i] = i < vis[0] ? sc : -INFINITY;
+      } else {
+        const float *wu = sw[upar];
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+          uint32_t d[N1];
+#pragma unroll
+          for (int c = 0; c < N1 / 16; ++c) tmem_ld16(taddr + g * N1 + 16 * c, d + 16 * c);
+          tmem_wait_ld_regs<N1>(d);
+          float sc = 0.f;
+#pragma unroll
+          for (int h = 0; h < N1; ++h) sc = fmaf(wu[g * N1 + h], fmaxf(__uint_as_float(d[h]), 0.f), sc);
+          if (g < nrows && i < a.nc_max) {
+            if (i < vis[g]) a.scores[(size_t)(r0 + g) * a.nc_max + i] = sc;
+            else if (a.fill_invisible) a.scores[(size_t)(r0 + g) * a.nc_max + i] = -INFINITY;
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(t_empty + 8 * acc);
+      }
       ++nt;
     }
     // -inf past each row's visible tiles (rows split over the CTAs)

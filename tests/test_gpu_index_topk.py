@@ -86,6 +86,28 @@ def test_bf16_head_and_dim_shapes(HI, dI):
     check_all(qI, w, kI, lens, 200, "bf16", q_pos=q_pos)
 
 
+@pytest.mark.parametrize("HI,dI", [(16, 128), (32, 64), (64, 128), (128, 64)])
+def test_grouped_query_rows(HI, dI):
+    """Several query rows of a sequence share each key tile (units of up to
+    four rows): 7 rows per sequence (a partial last unit whose query block
+    reaches into the next sequence's rows), two sequences of different
+    lengths, positions out of order; scores of every row (-inf where not
+    visible) and the selections checked."""
+    seed = 2000 + HI + dI
+    B, Tq, nc = 2, 7, 3000
+    lens = np.array([4 * nc, 4 * nc - 5001], np.int32)
+    q_pos = np.array([[11999, 20, 3, 7000, 4, 11998, 5555],
+                      [6998, 0, 6000, 129, 131, 6997, 2]], np.int32)
+    qI = W.normal(seed, "qI", (B, Tq, HI, dI), 1.0, "bf16")
+    w = W.normal(seed, "w", (B, Tq, HI), 1.0 / HI, "bf16")
+    kI = W.normal(seed, "kI", (B, nc, dI), 1.0, "bf16")
+    idx, sc = check_all(qI, w, kI, lens, 300, "bf16", q_pos=q_pos)
+    vis = oracle.visible(lens, B, Tq, 4, q_pos)
+    for b in range(B):
+        for tq in range(Tq):
+            assert np.all(np.isneginf(sc[b, tq, vis[b, tq]:]))
+
+
 def test_causal_rows_prefill_like():
     """Many query rows at increasing positions (v from 0 to > k): visibility
     and the v <= k / v == 0 paths."""
