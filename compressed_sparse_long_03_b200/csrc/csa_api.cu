@@ -421,16 +421,26 @@ int launch_index_tc_n(const void *qI, const void *w, const void *kI, const int32
   return launch_index_tc<128, 1, DI>(qI, w, kI, lens, q_pos, R, Tq, HI, nc_max, scores, fill, st);
 }
 
+template <int CS, int NT>
+int launch_topk_nt(const float *scores, const int32_t *lens, const int32_t *q_pos, int R,
+                   int Tq, int nc_max, int k, int32_t *idx_out, cudaStream_t st) {
+  const int per = (nc_max + CS - 1) / CS;
+  const size_t smem = csa::topk_dyn_bytes(per > 0 ? per : 1);
+  auto kern = csa::k_topk<CS, NT>;
+  int rc = ensure_smem(kern, smem, "csa_index_topk");
+  if (rc) return rc;
+  return launch_cluster(kern, CS, (unsigned)CS * R, NT, smem, st, "csa_index_topk (select)", scores,
+                        lens, q_pos, Tq, nc_max, k, idx_out);
+}
+
+// Rows of up to 4096 keys per CTA take 256-thread CTAs (several per SM);
+// longer slices 1024 threads.
 template <int CS>
 int launch_topk(const float *scores, const int32_t *lens, const int32_t *q_pos, int R,
                 int Tq, int nc_max, int k, int32_t *idx_out, cudaStream_t st) {
-  const int per = (nc_max + CS - 1) / CS;
-  const size_t smem = csa::topk_dyn_bytes(per > 0 ? per : 1);
-  auto kern = csa::k_topk<CS>;
-  int rc = ensure_smem(kern, smem, "csa_index_topk");
-  if (rc) return rc;
-  return launch_cluster(kern, CS, (unsigned)CS * R, csa::kTopkThreads, smem, st,
-                        "csa_index_topk (select)", scores, lens, q_pos, Tq, nc_max, k, idx_out);
+  if ((nc_max + CS - 1) / CS <= 4096)
+    return launch_topk_nt<CS, 256>(scores, lens, q_pos, R, Tq, nc_max, k, idx_out, st);
+  return launch_topk_nt<CS, csa::kTopkThreads>(scores, lens, q_pos, R, Tq, nc_max, k, idx_out, st);
 }
 
 // Whether this device can co-schedule a 16-CTA cluster of the top-k kernel

@@ -117,16 +117,19 @@ __device__ __forceinline__ void find_bucket(TopkShared &sh, int n, int need, int
   __syncthreads();
 }
 
-// idx_out row r: the k selected visible entries, ascending.
-template <int CS>
-__global__ void __launch_bounds__(kTopkThreads) k_topk(const float *__restrict__ scores,
+// idx_out row r: the k selected visible entries, ascending.  NT threads per
+// CTA (1024 for long rows; 256 for short ones, so that several CTAs share an
+// SM).
+template <int CS, int NT = kTopkThreads>
+__global__ void __launch_bounds__(NT) k_topk(const float *__restrict__ scores,
                                                        const int32_t *__restrict__ lens,
                                                        const int32_t *__restrict__ q_pos, int Tq,
                                                        int nc_max, int k,
                                                        int32_t *__restrict__ idx_out) {
   extern __shared__ uint32_t dyn[];
   __shared__ TopkShared sh;
-  constexpr int NT = kTopkThreads, NW = NT / 32;
+  static_assert(NT >= 256 && kScoreBins % NT == 0, "256-bucket searches need 256 threads");
+  constexpr int NW = NT / 32;
   const int rank = (CS > 1) ? (int)cg::this_cluster().block_rank() : 0;
   const int r = blockIdx.x / CS;  // clusters tile the grid along x
   const int b = r / Tq, tq = r % Tq;
