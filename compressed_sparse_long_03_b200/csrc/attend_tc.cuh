@@ -41,8 +41,12 @@ constexpr uint32_t kAtQAtom = 128 * 128;             // 128 rows x 128 B
 constexpr uint32_t kAtKHalf = kAtMaxTile * 128;      // one 64-wide d slice of the key tile
 constexpr uint32_t kAtPAtom = 128 * 128;             // 128 heads x 64 keys x 2 B
 constexpr uint32_t kAtPart = 128 * 128 * 4;          // partial outputs pushed by the cluster
-constexpr size_t kAtSmem =
-    1024 + 2 * kAtQAtom + 2 * kAtKHalf + (kAtMaxTile / 64) * kAtPAtom + kAtPart;
+// Dynamic shared memory: Q, the key tile (two, double-buffered, for one-CTA
+// rows), P, and for clusters the partials pushed by the peers.
+__host__ __device__ constexpr size_t at_smem_bytes(int cs) {
+  return 1024 + 2 * kAtQAtom + (cs == 1 ? 2 : 1) * 2 * kAtKHalf + (kAtMaxTile / 64) * kAtPAtom +
+         (cs == 1 ? 0 : kAtPart);
+}
 
 template <int CS>
 __global__ void __launch_bounds__(kAtThreads, 1) k_attend_tc(AttendArgs a) {
@@ -51,8 +55,9 @@ __global__ void __launch_bounds__(kAtThreads, 1) k_attend_tc(AttendArgs a) {
   extern __shared__ uint8_t smem_raw[];
   __shared__ uint32_t tmem_holder;
   __shared__ uint64_t bar_s, bar_o;
-  __shared__ int kvalid[kAtMaxTile / 32];  // validity bits, one word per 32 keys
-  __shared__ const __nv_bfloat16 *rowp[kAtMaxTile];
+  constexpr int NKB = CS == 1 ? 2 : 1;  // key-tile buffers
+  __shared__ int kvalid[NKB][kAtMaxTile / 32];  // validity bits, one word per 32 keys
+  __shared__ const __nv_bfloat16 *rowp[NKB][kAtMaxTile];
   __shared__ float pm[136], pl[136];   // pushed partial max / sum [hl * CS + c]
   __shared__ float xmax[2][128];       // per-half row max (then sum) of the partner
   __shared__ float mw[136], minv[128];  // merge weights [hl * CS + c], 1 / sum
@@ -61,8 +66,8 @@ __global__ void __launch_bounds__(kAtThreads, 1) k_attend_tc(AttendArgs a) {
   uint8_t *base = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t *sQ = base;
-  uint8_t *sK = sQ + 2 * kAtQAtom;
-  uint8_t *sP = sK + 2 * kAtKHalf;
+  uint8_t *sK = sQ + 2 * kAtQAtom;       // NKB x [2 d-halves][kAtMaxTile rows][128 B]
+  uint8_t *sP = sK + NKB * 2 * kAtKHalf;
   // partials of the heads this CTA finalises, written by every CTA of the
   // cluster: [head slot hl][source rank c][128] (slot hl = head h / CS)
   float *part = reinterpret_cast<float *>(sP + (kAtMaxTile / 64) * kAtPAtom);
@@ -150,15 +155,14 @@ __global__ void __launch_bounds__(kAtThreads, 1) k_attend_tc(AttendArgs a) {
   uint32_t ns = 0, no = 0;
   bool alive = true;
 
-  for (int p0 = lo; p0 < hi && alive; p0 += kAtMaxTile) {
-    const int ntile = min(kAtMaxTile, hi - p0);
-    const int nchunk = (ntile + 31) >> 5;  // 32-key chunks; MMA N = 32 * nchunk
-    // ---- row pointers of the tile's keys (one coalesced index read), then
-    // the rows themselves: 16 chunks of 16 B each, no dependent global loads
-    for (int j = tid; j < nchunk * 32; j += kAtThreads) {
+  // row pointers (one coalesced index read) and validity words of the tile
+  // at p0 into buffer kb
+  auto stage_ptrs = [&](int p0, int kb) {
+    const int nt = min(kAtMaxTile, hi - p0), nc = (nt + 31) >> 5;
+    for (int j = tid; j < nc * 32; j += kAtThreads) {
       const int p = p0 + j;
       const __nv_bfloat16 *row = nullptr;
-      if (j < ntile) {
+      if (j < nt) {
         if (p < nsel) {
           const int i = a.idx ? __ldg(a.idx + (size_t)r * a.k + p) : p;
           if (i >= 0 && i < v) row = kv_c + ((size_t)b * a.nc_max + i) * D;
@@ -167,23 +171,54 @@ __global__ void __launch_bounds__(kAtThreads, 1) k_attend_tc(AttendArgs a) {
           row = kv_tok + ((size_t)b * a.n_tok + (s % a.n_tok)) * D;
         }
       }
-      rowp[j] = row;
+      rowp[kb][j] = row;
       // a warp covers 32 consecutive keys: one validity word per 32
       const unsigned vm = __ballot_sync(0xffffffffu, row != nullptr);
-      if ((tid & 31) == 0) kvalid[j >> 5] = (int)vm;
+      if ((tid & 31) == 0) kvalid[kb][j >> 5] = (int)vm;
     }
-    __syncthreads();
-    for (int u = tid; u < nchunk * 32 * 16; u += kAtThreads) {
+  };
+  // the tile's rows into key buffer kb: 16 chunks of 16 B each (one
+  // cp.async group)
+  auto gather = [&](int p0, int kb) {
+    const int nt = min(kAtMaxTile, hi - p0), nc = (nt + 31) >> 5;
+    const uint32_t k0 = smem_u32(sK) + kb * 2 * kAtKHalf;
+    for (int u = tid; u < nc * 32 * 16; u += kAtThreads) {
       const int j = u >> 4, c = u & 15;
-      const __nv_bfloat16 *row = rowp[j];
-      const uint32_t dst = smem_u32(sK) + (c >> 3) * kAtKHalf + j * 128 + (((c & 7) ^ (j & 7)) << 4);
-      cp_async16(dst, row ? row + c * 8 : kv_tok, row ? 16u : 0u);
+      const __nv_bfloat16 *row = rowp[kb][j];
+      cp_async16(k0 + (c >> 3) * kAtKHalf + j * 128 + (((c & 7) ^ (j & 7)) << 4), row ? row + c * 8 : kv_tok,
+                 row ? 16u : 0u);
     }
-    cp_async_wait_all();
+    cp_async_commit();
+  };
+  if constexpr (NKB == 2) {
+    if (lo < hi) {
+      stage_ptrs(lo, 0);
+      __syncthreads();
+      gather(lo, 0);
+    }
+  }
+
+  int kb = 0;
+  for (int p0 = lo; p0 < hi && alive; p0 += kAtMaxTile, kb ^= NKB - 1) {
+    const int ntile = min(kAtMaxTile, hi - p0);
+    const int nchunk = (ntile + 31) >> 5;  // 32-key chunks; MMA N = 32 * nchunk
+    const int pn = p0 + kAtMaxTile;
+    if constexpr (NKB == 1) {
+      stage_ptrs(p0, 0);
+      __syncthreads();
+      gather(p0, 0);
+    } else if (pn < hi) {
+      stage_ptrs(pn, kb ^ 1);  // while this tile's rows are in flight
+    }
+    cp_async_wait_group<0>();
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    if constexpr (NKB == 2) {
+      if (pn < hi) gather(pn, kb ^ 1);  // the next tile's rows during this tile's math
+    }
+    const uint32_t sKb = smem_u32(sK) + kb * 2 * kAtKHalf;
     // ---- S = Q K^T
     if (tid == 0) {
       const uint32_t idesc = idesc_bf16_f32(128, 32 * nchunk);
@@ -191,8 +226,7 @@ __global__ void __launch_bounds__(kAtThreads, 1) k_attend_tc(AttendArgs a) {
       for (int k = 0; k < D / 16; ++k) {
         const uint32_t off = (k >> 2) * kAtQAtom + (k & 3) * 32;
         const uint32_t koff = (k >> 2) * kAtKHalf + (k & 3) * 32;
-        umma_bf16(tS, sdesc_kmajor_sw128(smem_u32(sQ) + off), sdesc_kmajor_sw128(smem_u32(sK) + koff),
-                  idesc, k > 0);
+        umma_bf16(tS, sdesc_kmajor_sw128(smem_u32(sQ) + off), sdesc_kmajor_sw128(sKb + koff), idesc, k > 0);
       }
       umma_commit(smem_u32(&bar_s));
     }
@@ -222,7 +256,7 @@ __global__ void __launch_bounds__(kAtThreads, 1) k_attend_tc(AttendArgs a) {
         if (c0 + i < c1) {
 #pragma unroll
           for (int jj = 0; jj < 32; ++jj) asm volatile("" : "+r"(sv[i][jj]));
-          const uint32_t vm = (uint32_t)kvalid[c0 + i];
+          const uint32_t vm = (uint32_t)kvalid[kb][c0 + i];
 #pragma unroll
           for (int jj = 0; jj < 32; ++jj)
             if ((vm >> jj) & 1u) mt = fmaxf(mt, __uint_as_float(sv[i][jj]) * a.scale_log2);
@@ -240,7 +274,7 @@ __global__ void __launch_bounds__(kAtThreads, 1) k_attend_tc(AttendArgs a) {
       for (int i = 0; i < kAtMaxTile / 64; ++i) {
         if (c0 + i < c1) {
           const int c = c0 + i;
-          const uint32_t vm = (uint32_t)kvalid[c];
+          const uint32_t vm = (uint32_t)kvalid[kb][c];
 #pragma unroll
           for (int g = 0; g < 4; ++g) {  // 8 keys -> one 16-byte chunk of P
             uint32_t pk[4];
@@ -278,7 +312,7 @@ __global__ void __launch_bounds__(kAtThreads, 1) k_attend_tc(AttendArgs a) {
       for (int k = 0; k < 2 * nchunk; ++k) {  // 16 keys per MMA
         const uint32_t poff = (k >> 2) * kAtPAtom + (k & 3) * 32;
         umma_bf16(tO, sdesc_kmajor_sw128(smem_u32(sP) + poff),
-                  sdesc_mnmajor_sw128(smem_u32(sK) + k * 2048, kAtKHalf), idesc, k > 0);
+                  sdesc_mnmajor_sw128(sKb + k * 2048, kAtKHalf), idesc, k > 0);
       }
       umma_commit(smem_u32(&bar_o));
     }
@@ -299,13 +333,38 @@ __global__ void __launch_bounds__(kAtThreads, 1) k_attend_tc(AttendArgs a) {
     tc_fence_before();
     __syncthreads();  // every lane done with S, P and O before they are rewritten
   }
+  cp_async_wait_group<0>();  // a tile still in flight after a timeout lands before exit
 
+  xmax[half][hrow] = l_run;
+  __syncthreads();
+  if constexpr (CS == 1) {
+    // one CTA holds the whole row: normalise (with the sink when given) and
+    // store this half's 64 output columns
+    if (hrow < H) {
+      const float lt = l_run + xmax[half ^ 1][hrow];
+      const float sk = sink_log2(a, hrow);
+      float f = 1.f / lt;
+      if (sk != -INFINITY) {
+        const float M = fmaxf(m_run, sk), so = ex2(m_run - M);
+        f = so / (lt * so + ex2(sk - M));
+      }
+      uint4 *dst = reinterpret_cast<uint4 *>(out + (size_t)hrow * D + half * (D / 2));
+#pragma unroll
+      for (int j = 0; j < D / 16; ++j) {
+        uint32_t w4[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          __nv_bfloat162 pr = __floats2bfloat162_rn(o[8 * j + 2 * e] * f, o[8 * j + 2 * e + 1] * f);
+          w4[e] = *reinterpret_cast<uint32_t *>(&pr);
+        }
+        dst[j] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+      }
+    }
+  } else {
   // ---- push this CTA's partial (max, sum, output) of head h into the CTA
   // that finalises h (rank h % CS), one cluster barrier, merge locally; the
   // two halves of a row push their output columns, half 0 the max and the
   // sum of both halves
-  xmax[half][hrow] = l_run;
-  __syncthreads();
   if (hrow < H) {
     const int own = hrow % CS, slot = (hrow / CS) * CS + rank;
     float4 *dst = reinterpret_cast<float4 *>(att_peer<CS>(part, own) + (size_t)slot * D + half * (D / 2));
@@ -357,6 +416,7 @@ __global__ void __launch_bounds__(kAtThreads, 1) k_attend_tc(AttendArgs a) {
     pk.y = *reinterpret_cast<uint32_t *>(&hi2);
     *reinterpret_cast<uint2 *>(out + (size_t)h * D + 4 * j) = pk;
   }
+  }  // clusters
   if (tid == 0 && abort_flag) raise_dev_err(kDevErrTimeout);
   tc_fence_before();
   __syncthreads();

@@ -512,9 +512,10 @@ int launch_attend_tc(const csa::AttendArgs &a, int R, cudaStream_t st, const cha
     case 4: kern = csa::k_attend_tc<4>; break;
     default: kern = csa::k_attend_tc<8>; break;
   }
-  int rc = ensure_smem(kern, csa::kAtSmem, what);
+  const size_t smem = csa::at_smem_bytes(cs);
+  int rc = ensure_smem(kern, smem, what);
   if (rc) return rc;
-  return launch_cluster(kern, cs, (unsigned)cs * R, csa::kAtThreads, csa::kAtSmem, st, what, a);
+  return launch_cluster(kern, cs, (unsigned)cs * R, csa::kAtThreads, smem, st, what, a);
 }
 
 int attend_common(const void *q, const void *kv_c, const void *kv_tok, int n_tok,
