@@ -54,6 +54,8 @@ def _load():
         lib.orc_select_topk.argtypes = [P, P, L, I, I, P]
         lib.orc_visible.argtypes = [P, P, I, I, I, P]
         lib.orc_attend.argtypes = [P, P, P, I, P, P, P, I, I, I, I, I, I, I, I, D, P, I, P]
+        lib.orc_quantize_mxfp4.argtypes = [P, I, L, I, P, P]
+        lib.orc_dequant_mxfp4.argtypes = [P, P, L, I, P]
         lib.orc_set_threads.argtypes = [I]
         lib.orc_get_threads.restype = I
         for name in ("orc_round", "orc_csa_compress", "orc_hca_compress", "orc_index_scores",
@@ -237,4 +239,31 @@ def attend(q, kv_c, kv_tok, lens, idx=None, q_pos=None, window=128, m=4, scale=0
     _check(lib.orc_attend(pq, pc if nc_max else None, pt, n_tok, pi, pl, pp, B, Tq, H, d,
                           nc_max, k, window, m, float(scale), ps, dt,
                           out.ctypes.data_as(ctypes.c_void_p)), "attend")
+    return out
+
+
+def quantize_mxfp4(k):
+    """MXFP4 indexer keys: k [..., dI] (float32 or bf16 bits) -> (codes
+    uint8 [..., dI/2], scales uint8 [..., dI/32])."""
+    lib = _load()
+    dt = _dt_of(k)
+    k, pk = _c(k)
+    dI = k.shape[-1]
+    rows = k.size // dI
+    codes = np.empty(k.shape[:-1] + (dI // 2,), np.uint8)
+    scales = np.empty(k.shape[:-1] + (dI // 32,), np.uint8)
+    _check(lib.orc_quantize_mxfp4(pk, dt, rows, dI, codes.ctypes.data_as(ctypes.c_void_p),
+                                  scales.ctypes.data_as(ctypes.c_void_p)), "quantize_mxfp4")
+    return codes, scales
+
+
+def dequant_mxfp4(codes, scales):
+    """(codes, scales) -> float64 [..., dI], the exact key values."""
+    lib = _load()
+    codes, pc = _c(codes, np.uint8)
+    scales, ps = _c(scales, np.uint8)
+    dI = codes.shape[-1] * 2
+    rows = codes.size // (dI // 2)
+    out = np.empty(codes.shape[:-1] + (dI,), np.float64)
+    _check(lib.orc_dequant_mxfp4(pc, ps, rows, dI, out.ctypes.data_as(ctypes.c_void_p)), "dequant_mxfp4")
     return out

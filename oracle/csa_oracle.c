@@ -493,3 +493,84 @@ int orc_attend(const void *q, const void *kv_c, const void *kv_tok, int n_tok,
   }
   return err;
 }
+
+/* ------------------------------------------------------------------ */
+/* MXFP4 indexer keys                                                 */
+/* ------------------------------------------------------------------ */
+/*
+ * [A4] "The KV cache, recomputed": the indexer key is 128 numbers in FP4
+ * with one one-byte scale per 32 (68 bytes); CSA bullet: the indexer runs in
+ * FP4.  Reading (the OCP microscaling format, the pages naming the sizes
+ * only): each block of 32 consecutive elements of a key shares a power-of-
+ * two scale 2^X stored as the byte X + 127; each element is an E2M1 code
+ * (sign bit 3; magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6 for codes 0..7), two per
+ * byte, element 2j in the low nibble.  Quantisation: X = floor(log2 amax) - 2
+ * (amax the block's largest magnitude; the largest E2M1 magnitude 6 has
+ * exponent 2), clamped to [-127, 127], X = -127 for an all-zero block; each
+ * element becomes the nearest magnitude of x / 2^X, ties to the even code,
+ * saturating at 6.  Dequantised value: sign * magnitude(code) * 2^X.
+ * The score of a query against such a key is the indexer score of
+ * orc_index_scores against the dequantised key.
+ */
+static const double kE2M1[8] = {0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0};
+
+/* nearest E2M1 magnitude code of y >= 0, ties to the even code */
+static int e2m1_code(double y) {
+  if (y >= 6.0) return 7;
+  int lo = 0;
+  while (lo < 7 && kE2M1[lo + 1] <= y) ++lo;
+  if (kE2M1[lo] == y || lo == 7) return lo;
+  const double dlo = y - kE2M1[lo], dhi = kE2M1[lo + 1] - y;
+  if (dlo < dhi) return lo;
+  if (dhi < dlo) return lo + 1;
+  return (lo % 2 == 0) ? lo : lo + 1;
+}
+
+/* k: [rows][dI] (bf16 or fp32), codes: [rows][dI/2], scales: [rows][dI/32] */
+int orc_quantize_mxfp4(const void *k, int dt, long rows, int dI, uint8_t *codes, uint8_t *scales) {
+  if (!k || !codes || !scales || rows < 0 || dI <= 0 || dI % 32) return ORC_ERR_ARG;
+  if (dt != ORC_F32 && dt != ORC_BF16) return ORC_ERR_ARG;
+#pragma omp parallel for schedule(static)
+  for (long r = 0; r < rows; ++r) {
+    for (int blk = 0; blk < dI / 32; ++blk) {
+      double amax = 0.0;
+      for (int e = 0; e < 32; ++e) {
+        const double x = fabs(ld(k, dt, (size_t)r * dI + blk * 32 + e));
+        if (x > amax) amax = x;
+      }
+      int X = -127;
+      if (amax > 0.0) {
+        int ex;
+        (void)frexp(amax, &ex);  /* amax = f * 2^ex, 0.5 <= f < 1: floor(log2 amax) = ex - 1 */
+        X = ex - 1 - 2;
+        if (X < -127) X = -127;
+        if (X > 127) X = 127;
+      }
+      scales[(size_t)r * (dI / 32) + blk] = (uint8_t)(X + 127);
+      for (int e = 0; e < 32; e += 2) {
+        uint8_t byte = 0;
+        for (int h = 0; h < 2; ++h) {
+          const double x = ld(k, dt, (size_t)r * dI + blk * 32 + e + h);
+          int c = e2m1_code(ldexp(fabs(x), -X));
+          if (signbit(x)) c |= 8;
+          byte |= (uint8_t)(c << (4 * h));
+        }
+        codes[(size_t)r * (dI / 2) + (blk * 32 + e) / 2] = byte;
+      }
+    }
+  }
+  return ORC_OK;
+}
+
+/* codes/scales as above -> out [rows][dI] double (exact values) */
+int orc_dequant_mxfp4(const uint8_t *codes, const uint8_t *scales, long rows, int dI, double *out) {
+  if (!codes || !scales || !out || rows < 0 || dI <= 0 || dI % 32) return ORC_ERR_ARG;
+  for (long r = 0; r < rows; ++r)
+    for (int e = 0; e < dI; ++e) {
+      const int c = (codes[(size_t)r * (dI / 2) + e / 2] >> (4 * (e & 1))) & 15;
+      const int X = (int)scales[(size_t)r * (dI / 32) + e / 32] - 127;
+      const double v = ldexp(kE2M1[c & 7], X);
+      out[(size_t)r * dI + e] = (c & 8) ? -v : v;
+    }
+  return ORC_OK;
+}

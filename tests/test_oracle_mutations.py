@@ -16,7 +16,8 @@ import pytest
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 SRC = os.path.join(ROOT, "oracle", "csa_oracle.c")
 PINS = ["tests/test_oracle_compress.py", "tests/test_oracle_index_topk.py",
-        "tests/test_oracle_attend.py", "tests/test_oracle_e2e.py"]
+        "tests/test_oracle_attend.py", "tests/test_oracle_e2e.py",
+        "tests/test_oracle_mxfp4.py"]
 
 MUTANTS = {
     "csa_series_swapped": ("const void *W = (j < 4) ? Wa : Wb;", "const void *W = (j < 4) ? Wb : Wa;"),
@@ -41,6 +42,8 @@ MUTANTS = {
     "attend_visibility": ("long vis = (t + 1) / m;", "long vis = (t + 2) / m;"),
     "attend_invisible_index_used": ("if (i < 0 || i >= vis) continue;", "if (i < 0 || i >= nc_max) continue;"),
     "attend_sink_ignored": ("if (sink) den += exp(sink[h] - mx);", ""),
+    "mxfp4_ties_to_odd": ("return (lo % 2 == 0) ? lo : lo + 1;", "return (lo % 2 == 1) ? lo : lo + 1;"),
+    "mxfp4_scale_off_by_one": ("X = ex - 1 - 2;", "X = ex - 1 - 1;"),
     "round_double_rounding": ("r = nearbyint(ldexp(a, -q));", "r = nearbyint(ldexp((double)(float)a, -q));"),
 }
 
