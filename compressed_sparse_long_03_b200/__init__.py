@@ -66,11 +66,13 @@ def lib() -> ctypes.CDLL:
         L.csa_index_topk_noalloc_max_elems.argtypes = []
         L.csa_index_topk_noalloc_max_elems.restype = S
         L.csa_index_scores.argtypes = [P, P, P, P, P, I, I, I, I, I, I, P, P]
+        L.csa_quantize_mxfp4.argtypes = [P, I, I, I, I, P, P, P]
+        L.csa_index_topk_mxfp4.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, P, P, P, S, P]
         L.csa_topk.argtypes = [P, P, P, I, I, I, I, P, P]
         L.csa_attend.argtypes = [P, P, P, I, P, P, P, I, I, I, I, I, I, I, F, P, I, P, P]
         L.hca_attend.argtypes = [P, P, P, I, P, P, I, I, I, I, I, I, I, F, P, I, P, P]
         for name in ("csa_check_device_error", "csa_compress", "hca_compress", "csa_compress_step",
-                     "hca_compress_step", "csa_index_topk",
+                     "hca_compress_step", "csa_quantize_mxfp4", "csa_index_topk_mxfp4", "csa_index_topk",
                      "csa_index_topk_noalloc", "csa_index_scores", "csa_topk", "csa_attend", "hca_attend"):
             getattr(L, name).restype = I
         _lib = L
@@ -226,6 +228,42 @@ def csa_index_topk_noalloc(q_idx, w, k_idx, lens, k, idx_out, q_pos=None, stream
         raise ValueError("idx_out must be an int32 tensor of shape [B][Tq][k]")
     _check(lib().csa_index_topk_noalloc(_p(q_idx), _p(w), _p(k_idx), _i32(lens), _i32(q_pos), B, Tq,
                                         HI, dI, nc_max, k, _dt(q_idx), _i32(idx_out), _s(stream)))
+    return idx_out
+
+
+def _u8(t):
+    if t is not None and t.dtype != torch.uint8:
+        raise TypeError("codes and scales are uint8")
+    return _p(t)
+
+
+def csa_quantize_mxfp4(k_idx, codes=None, scales=None, stream=None):
+    """Indexer keys [B][nc_max][dI] (bf16 or fp32) -> MXFP4 (codes uint8
+    [B][nc_max][dI/2], scales uint8 [B][nc_max][dI/32])."""
+    B, nc, dI = k_idx.shape
+    if codes is None:
+        codes = torch.empty(B, nc, dI // 2, dtype=torch.uint8, device=k_idx.device)
+    if scales is None:
+        scales = torch.empty(B, nc, dI // 32, dtype=torch.uint8, device=k_idx.device)
+    _check(lib().csa_quantize_mxfp4(_p(k_idx), B, nc, dI, _dt(k_idx), _u8(codes), _u8(scales), _s(stream)))
+    return codes, scales
+
+
+def csa_index_topk_mxfp4(q_idx, w, codes, scales, lens, k, q_pos=None, idx_out=None, scores_out=None,
+                         workspace=None, stream=None):
+    """csa_index_topk over an MXFP4 indexer-key cache (codes [B][nc_max][dI/2],
+    scales [B][nc_max][dI/32]); q_idx and w bf16."""
+    B, Tq, HI, dI = q_idx.shape
+    nc_max = codes.shape[1]
+    if idx_out is None:
+        idx_out = torch.empty(B, Tq, k, dtype=torch.int32, device=q_idx.device)
+    need = index_topk_workspace_size(B, Tq, nc_max, scores_out is not None)
+    if workspace is None and need:
+        workspace = index_topk_workspace(B, Tq, nc_max, scores_out is not None, q_idx.device)
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check(lib().csa_index_topk_mxfp4(_p(q_idx), _p(w), _u8(codes), _u8(scales), _i32(lens), _i32(q_pos),
+                                      B, Tq, HI, dI, nc_max, k, _i32(idx_out), _p(scores_out),
+                                      _p(workspace), ws_bytes, _s(stream)))
     return idx_out
 
 

@@ -23,6 +23,7 @@
 #include "compress.cuh"
 #include "compress_tc.cuh"
 #include "compress_step.cuh"
+#include "mxfp4.cuh"
 #include "index_score_fma.cuh"
 #include "index_score_tc.cuh"
 #include "topk.cuh"
@@ -196,6 +197,22 @@ int encode_bf16_2d(CUtensorMap *map, const void *base, uint64_t inner, uint64_t 
   CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides,
                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(CSA_ERR_CUDA, "%s: tensor map encoding failed (%d)", what, (int)r);
+  return CSA_OK;
+}
+
+// 2-D byte tensor [outer][inner], box [box_outer][box_inner], no swizzle.
+int encode_u8_2d(CUtensorMap *map, const void *base, uint64_t inner, uint64_t outer, uint32_t box_inner,
+                 uint32_t box_outer, const char *what) {
+  encode_tiled_fn enc = get_encode_tiled();
+  if (!enc) return fail(CSA_ERR_CUDA, "%s: cuTensorMapEncodeTiled is unavailable", what);
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {inner};
+  const cuuint32_t box[2] = {box_inner, box_outer};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(CSA_ERR_CUDA, "%s: tensor map encoding failed (%d)", what, (int)r);
   return CSA_OK;
 }
@@ -419,6 +436,51 @@ int launch_index_tc_n(const void *qI, const void *w, const void *kI, const int32
   if (HI <= 32) return launch_index_tc<32, 1, DI>(qI, w, kI, lens, q_pos, R, Tq, HI, nc_max, scores, fill, st);
   if (HI <= 64) return launch_index_tc<64, 1, DI>(qI, w, kI, lens, q_pos, R, Tq, HI, nc_max, scores, fill, st);
   return launch_index_tc<128, 1, DI>(qI, w, kI, lens, q_pos, R, Tq, HI, nc_max, scores, fill, st);
+}
+
+// Indexer scores over an MXFP4 key cache (one query row per unit).
+template <int N, int DI>
+int launch_index_fp4(const void *qI, const void *w, const uint8_t *codes, const uint8_t *scales,
+                     const int32_t *lens, const int32_t *q_pos, int R, int Tq, int HI, int nc_max,
+                     float *scores, bool fill, cudaStream_t st) {
+  const char *what = "csa_index_topk_mxfp4";
+  CUtensorMap tmC, tmQ;
+  const int B = R / Tq;
+  int rc = encode_u8_2d(&tmC, codes, DI / 2, (uint64_t)B * nc_max, DI / 2, csa::kTcRows, what);
+  if (rc) return rc;
+  rc = encode_bf16_2d(&tmQ, qI, DI, (uint64_t)R * HI, 64, N, what);
+  if (rc) return rc;
+  constexpr size_t A_STAGE = (size_t)csa::kTcRows * DI * 2, C_STAGE = (size_t)csa::kTcRows * DI / 2,
+                   B_SLOT = (size_t)N * DI * 2;
+  const size_t smem = 1024 + 3 * A_STAGE + 2 * B_SLOT + 6 * C_STAGE + 8 * (2 * 6 + 2 * 3 + 9);
+  auto kern = csa::k_index_score_fp4<N, DI>;
+  rc = ensure_smem(kern, smem, what);
+  if (rc) return rc;
+  csa::IndexTcArgs a;
+  a.w = static_cast<const __nv_bfloat16 *>(w);
+  a.lens = lens;
+  a.q_pos = q_pos;
+  a.scores = scores;
+  a.Tq = Tq;
+  a.HI = HI;
+  a.nc_max = nc_max;
+  a.R = R;
+  a.G = 1;
+  a.gpb = Tq;
+  a.U = R;
+  a.stages = 3;
+  a.fill_invisible = fill ? 1 : 0;
+  return launch_cluster(kern, 1, (unsigned)num_sms(), csa::kF4Threads, smem, st, what, tmC, tmQ, a, scales);
+}
+
+template <int DI>
+int launch_index_fp4_n(const void *qI, const void *w, const uint8_t *codes, const uint8_t *scales,
+                       const int32_t *lens, const int32_t *q_pos, int R, int Tq, int HI, int nc_max,
+                       float *scores, bool fill, cudaStream_t st) {
+  if (HI <= 16) return launch_index_fp4<16, DI>(qI, w, codes, scales, lens, q_pos, R, Tq, HI, nc_max, scores, fill, st);
+  if (HI <= 32) return launch_index_fp4<32, DI>(qI, w, codes, scales, lens, q_pos, R, Tq, HI, nc_max, scores, fill, st);
+  if (HI <= 64) return launch_index_fp4<64, DI>(qI, w, codes, scales, lens, q_pos, R, Tq, HI, nc_max, scores, fill, st);
+  return launch_index_fp4<128, DI>(qI, w, codes, scales, lens, q_pos, R, Tq, HI, nc_max, scores, fill, st);
 }
 
 template <int CS, int NT>
@@ -927,6 +989,71 @@ int csa_index_topk_noalloc(const void *q_idx, const void *w, const void *k_idx, 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   rc = index_scores_impl(q_idx, w, k_idx, lens, q_pos, B, Tq, HI, dI, nc_max, dt, scores, false, st);
   if (rc) return rc;
+  return topk_impl(scores, lens, q_pos, B, Tq, nc_max, k, idx_out, st);
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// MXFP4 indexer keys
+// ---------------------------------------------------------------------------
+extern "C" {
+
+int csa_quantize_mxfp4(const void *k_idx, int B, int nc_max, int dI, csa_dtype dt, uint8_t *codes,
+                       uint8_t *scales, void *stream) {
+  const char *what = "csa_quantize_mxfp4";
+  begin_call();
+  int rc = check_dtype(dt, what);
+  if (rc) return rc;
+  if (dI != 64 && dI != 128) return fail(CSA_ERR_UNSUPPORTED, "%s: dI=%d not in {64,128}", what, dI);
+  if (B < 0 || nc_max < 0) return fail(CSA_ERR_SHAPE, "%s: B, nc_max must be >= 0", what);
+  const long blocks = (long)B * nc_max * (dI / 32);
+  if (blocks == 0) return CSA_OK;
+  if (!k_idx || !codes || !scales) return fail(CSA_ERR_NULL, "%s: a required pointer is NULL", what);
+  if (!aligned16(k_idx) || !aligned16(codes)) return fail(CSA_ERR_ALIGN, "%s: keys and codes must be 16-byte aligned", what);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const unsigned grid = (unsigned)((blocks + 255) / 256);
+  if (dt == CSA_F32)
+    return launch_cluster(csa::k_quantize_mxfp4<float>, 1, grid, 256, 0, st, what,
+                          static_cast<const float *>(k_idx), blocks, codes, scales);
+  return launch_cluster(csa::k_quantize_mxfp4<__nv_bfloat16>, 1, grid, 256, 0, st, what,
+                        static_cast<const __nv_bfloat16 *>(k_idx), blocks, codes, scales);
+}
+
+int csa_index_topk_mxfp4(const void *q_idx, const void *w, const uint8_t *codes, const uint8_t *scales,
+                         const int32_t *lens, const int32_t *q_pos, int B, int Tq, int HI, int dI,
+                         int nc_max, int k, int32_t *idx_out, float *scores_out, void *workspace,
+                         size_t ws_bytes, void *stream) {
+  const char *what = "csa_index_topk_mxfp4";
+  begin_call();
+  int rc = check_index_args(what, CSA_BF16, B, Tq, HI, dI, nc_max);
+  if (rc) return rc;
+  if (dI != 64 && dI != 128) return fail(CSA_ERR_UNSUPPORTED, "%s: dI=%d not in {64,128}", what, dI);
+  rc = check_topk_args(what, B, Tq, nc_max, k);
+  if (rc) return rc;
+  if ((long)B * Tq == 0) return CSA_OK;
+  if (!q_idx || !w || !lens || !idx_out || (nc_max > 0 && (!codes || !scales)))
+    return fail(CSA_ERR_NULL, "%s: a required pointer is NULL", what);
+  if (!aligned16(q_idx) || !aligned16(w) || (codes && !aligned16(codes)) ||
+      (scales && (reinterpret_cast<uintptr_t>(scales) & 3)) || (scores_out && !aligned16(scores_out)))
+    return fail(CSA_ERR_ALIGN, "%s: tensors must be 16-byte aligned (scales 4-byte)", what);
+  const size_t need = csa_index_topk_workspace_size(B, Tq, nc_max, scores_out != nullptr);
+  if (need > 0 && (!workspace || ws_bytes < need))
+    return fail(CSA_ERR_WORKSPACE, "%s: workspace of %zu B needed, %zu given", what, need,
+                workspace ? ws_bytes : (size_t)0);
+  if (need > 0 && !aligned16(workspace)) return fail(CSA_ERR_ALIGN, "%s: workspace must be 16-byte aligned", what);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  float *scores = scores_out ? scores_out : static_cast<float *>(workspace);
+  const int R = B * Tq;
+  if (nc_max > 0) {
+    if ((long)B * nc_max >= (1L << 31) || (long)R * HI >= (1L << 31))
+      return fail(CSA_ERR_UNSUPPORTED, "%s: tensor too large for 32-bit coordinates", what);
+    rc = dI == 64 ? launch_index_fp4_n<64>(q_idx, w, codes, scales, lens, q_pos, R, Tq, HI, nc_max, scores,
+                                           scores_out != nullptr, st)
+                  : launch_index_fp4_n<128>(q_idx, w, codes, scales, lens, q_pos, R, Tq, HI, nc_max, scores,
+                                            scores_out != nullptr, st);
+    if (rc) return rc;
+  }
   return topk_impl(scores, lens, q_pos, B, Tq, nc_max, k, idx_out, st);
 }
 

@@ -246,6 +246,34 @@ CSA_API int csa_index_topk_noalloc(const void *q_idx, const void *w, const void 
                                    int32_t *idx_out, void *stream);
 
 /* ------------------------------------------------------------------------
+ * csa_quantize_mxfp4 / csa_index_topk_mxfp4 -- the indexer over FP4 keys.
+ *
+ * Anatomy page, "The KV cache, recomputed": the indexer key is 128 numbers
+ * in FP4 plus one byte of scale per 32 (68 bytes); CSA bullet: the lightning
+ * indexer runs in FP4.  Format (the OCP microscaling layout): per block of 32
+ * elements a power-of-two scale 2^X stored as the byte X + 127, X =
+ * floor(log2 amax) - 2 (-127 for an all-zero block); per element an E2M1
+ * code (sign bit 3; magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6: nearest to
+ * x / 2^X, ties to the even code, saturating at 6), two per byte, element 2j
+ * in the low nibble.
+ *   csa_quantize_mxfp4: k_idx [B][nc_max][dI] (bf16 or fp32) -> codes
+ *     [B][nc_max][dI/2] uint8, scales [B][nc_max][dI/32] uint8.
+ *   csa_index_topk_mxfp4: csa_index_topk with the key cache given as codes
+ *     and scales; the scores are those of csa_index_topk over the
+ *     dequantised keys (sign * magnitude * 2^X, each a bf16 number).  q_idx
+ *     and w bf16; codes 16-byte aligned, scales 4-byte aligned; other
+ *     arguments, workspace and selection as for csa_index_topk.
+ * Supported: dI in {64, 128}; HI in [1, 128].
+ * ---------------------------------------------------------------------- */
+CSA_API int csa_quantize_mxfp4(const void *k_idx, int B, int nc_max, int dI, csa_dtype dt, uint8_t *codes,
+                               uint8_t *scales, void *stream);
+
+CSA_API int csa_index_topk_mxfp4(const void *q_idx, const void *w, const uint8_t *codes,
+                                 const uint8_t *scales, const int32_t *lens, const int32_t *q_pos, int B,
+                                 int Tq, int HI, int dI, int nc_max, int k, int32_t *idx_out,
+                                 float *scores_out, void *workspace, size_t ws_bytes, void *stream);
+
+/* ------------------------------------------------------------------------
  * csa_attend -- sparse MQA attention over the selected entries + window.
  *
  * Anatomy page, "The skeleton": one key-value head is shared by every query
