@@ -46,9 +46,10 @@ def parse():
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-steps", type=int, default=1, help="oracle steps for cpu_baseline")
-    p.add_argument("--workload", type=int, default=4, choices=[1, 2, 3, 4, 5],
+    p.add_argument("--workload", type=int, default=4, choices=[1, 2, 3, 4, 5, 6],
                    help="4 (default): the 1M CSA decode step; 1, 2, 3, 5: the other "
-                        "workloads, one measurement line each (single GPU)")
+                        "workloads, one measurement line each (single GPU); 6: workload 4 "
+                        "with its indexer keys in MXFP4")
     return p.parse_args()
 
 
@@ -379,6 +380,23 @@ def other_workload_plan(wid, wl, csa, torch, D):
         byts = B * ((v + window) * d * 2 + 2 * H * d * 2)
         flops = 4.0 * B * (v + window) * H * d
         return stages, "queries/s", B, byts, flops, "one HCA decode step of the 32 sequences"
+    if wid == 6:
+        B, nc, H, d, dI, HI = s["B"], s["nc"], s["H"], s["d"], s["dI"], s["HI"]
+        codes, scales = csa.csa_quantize_mxfp4(D["kI"])
+        torch.cuda.synchronize()
+        idx = torch.empty(B, 1, k, dtype=torch.int32, device="cuda")
+        out = torch.empty(B, 1, H, d, dtype=torch.bfloat16, device="cuda")
+        ws = csa.index_topk_workspace(B, 1, nc, False)
+        stages = [
+            ("csa_index_topk_mxfp4", lambda: csa.csa_index_topk_mxfp4(D["qI"], D["w"], codes, scales, D["lens"],
+                                                                      k, idx_out=idx, workspace=ws)),
+            ("csa_attend", lambda: csa.csa_attend(D["q"], D["kv"], D["win"], idx, D["lens"], window=window,
+                                                  out=out)),
+        ]
+        byts = B * (nc * (dI // 2 + dI // 32) + (k + window) * d * 2 + (2 * H * d + HI * dI + HI) * 2)
+        flops = B * (2.0 * nc * HI * dI + 4.0 * (k + window) * H * d)
+        return stages, "queries/s", B, byts, flops, ("one decode step of the 1M workload with the indexer "
+                                                      "keys in MXFP4 (68 B per key): indexer + top-k, attention")
     if wid == 5:
         B, H, d, dI, HI, m = s["B"], s["H"], s["d"], s["dI"], s["HI"], s["m"]
         nc = s["nc"]
@@ -413,7 +431,7 @@ def run_other_workload(args):
     from tests.helpers import to_dev
     torch.cuda.set_device(0)
     wid = args.workload
-    wl = W.make(wid)
+    wl = W.make(4 if wid == 6 else wid)
     D = {n: to_dev(wl[n]) for n in wl.arrays if n != "needle_pos"}
     stages, unit, units, byts, flops, what = other_workload_plan(wid, wl, csa, torch, D)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
@@ -467,10 +485,11 @@ def run_other_workload(args):
     tfl = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     gbs = byts / (ms * 1e-3) / 1e9
     tfs = flops / (ms * 1e-3) / 1e12
-    line = {"metric": f"{wl.name}: {unit}", "value": units * 1000.0 / ms, "unit": unit, "n_gpus": 1,
+    name = "csa_decode_mxfp4keys_b4_n1048576" if wid == 6 else wl.name
+    line = {"metric": f"{name}: {unit}", "value": units * 1000.0 / ms, "unit": unit, "n_gpus": 1,
             "steps": K, "warmup": max(3, args.warmup), "ms_per_step": ms, "higher_is_better": True,
             "dtype": wl.dt, "data": "synthetic (seeded PCG64)",
-            "config": {"workload": wl.name, "step": what, "issue": how,
+            "config": {"workload": name, "step": what, "issue": how,
                        "l2": "flushed before every timed step (256 MiB write); events bracket the step"},
             "algorithmic": {"bytes_per_step": byts, "flops_per_step": flops, "achieved_gbs": gbs,
                             "frac_of_measured_hbm": gbs / hbm, "achieved_tflops": tfs,
@@ -524,6 +543,17 @@ def oracle_sample(wid, wl):
         return {"value": Tq / (tc + tr * Tq / rows), "unit": "tokens/s", "cores": cores, "kind": "oracle",
                 "sample": f"both compressors over the {n} tokens, then indexer + top-k + attention for "
                           f"{rows} of the {Tq} query rows (spread over the sequence), scaled to all rows"}
+    if wid == 6:
+        sl = slice(0, 1)
+
+        def one():
+            c, sc = oracle.quantize_mxfp4(wl["kI"][sl])
+            kdq = W.bf16_bits(oracle.dequant_mxfp4(c, sc).astype(np.float32))
+            idx, _ = oracle.index_topk(wl["qI"][sl], wl["w"][sl], kdq, wl["lens"][sl], k)
+            oracle.attend(wl["q"][sl], wl["kv"][sl], wl["win"][sl], wl["lens"][sl], idx=idx, window=window)
+        t = clock(one)
+        return {"value": 1.0 / t, "unit": "queries/s", "cores": cores, "kind": "oracle",
+                "sample": "one query of the batch (its keys quantised, dequantised, scored; attention)"}
     if wid == 3:
         nq = 4
         sl = slice(0, nq)

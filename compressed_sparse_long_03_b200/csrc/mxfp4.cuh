@@ -13,10 +13,11 @@
 // The scores over such a cache are exactly the bf16 indexer's scores over the
 // dequantised keys (every dequantised value is a bf16 number).  The decode
 // scan is HBM-bound, so the kernel streams the 68-byte keys and widens them
-// on chip: TMA brings 128-key code tiles (8 KB) into shared memory, four
-// converter warps expand each code byte through a 256-entry table (two bf16
-// values per byte) and apply the block's scale with one exact bf16x2
-// multiply, writing the 128-byte-swizzled bf16 tile that the MMA reads;
+// on chip: TMA brings 128-key code tiles (8 KB) into shared memory, two sets
+// of four converter warps (alternate tiles) expand each code byte through a
+// 256-entry table (two bf16 values per byte) and apply the block's scale
+// with one exact bf16x2 multiply, writing the 128-byte-swizzled bf16 tile
+// that the MMA reads;
 // producer, MMA issuer and epilogue are those of the bf16 kernel
 // (index_score_tc.cuh).  All waits are time-bounded.
 #pragma once
@@ -90,7 +91,7 @@ __global__ void __launch_bounds__(256) k_quantize_mxfp4(const T *__restrict__ k,
 // ---------------------------------------------------------------------------
 // indexer scores over MXFP4 keys
 // ---------------------------------------------------------------------------
-constexpr int kF4Threads = 320;  // producer, MMA, 4 epilogue warps, 4 converter warps
+constexpr int kF4Threads = 448;  // producer, MMA, 4 epilogue warps, 2 x 4 converter warps
 
 // bf16 pair of the two codes of byte b at scale 2^0 (low nibble in the low half)
 __host__ __device__ inline uint32_t e2m1_bf16(uint32_t c) {
@@ -319,18 +320,39 @@ __global__ void __launch_bounds__(kF4Threads, 1)
     // thread t widens key row t of the tile: its DI/2 code bytes (16-byte
     // chunks read in a rotated order against bank conflicts) and DI/32
     // scale bytes into 2*DI bytes of the swizzled bf16 tile
-    const int t = tid - 192;  // 0..127: the tile row
+    const int t = (tid - 192) & 127;      // the tile row
+    const uint32_t set = (tid - 192) >> 7;  // this set widens tiles nt % 2 == set
+    // the row's scale bytes (DI / 32 of them), loaded kPre own tiles ahead by
+    // a second cursor into a register ring (a load per tile would put a DRAM
+    // round trip in front of every tile)
+    constexpr int kPre = 8;
+    auto scale_word = [&](const TileWalk &w) -> uint32_t {
+      if (w.left <= 0 || w.j * kTcRows + t >= a.nc_max) return 0u;
+      const long key = (long)(w.r / a.Tq) * a.nc_max + (long)w.j * kTcRows + t;
+      if constexpr (DI == 128) return __ldg(reinterpret_cast<const uint32_t *>(scales) + key);
+      else return __ldg(reinterpret_cast<const uint16_t *>(scales) + key);
+    };
+    TileWalk ahead = wk;
+    if (set && ahead.left > 0) ahead.advance(a);  // this set's first tile
+    auto skip_other = [&](TileWalk &w) {          // to this set's next tile
+      for (int i = 0; i < 2 && w.left > 0; ++i) w.advance(a);
+    };
+    uint32_t ring[kPre];
+#pragma unroll
+    for (int i = 0; i < kPre; ++i) {
+      ring[i] = scale_word(ahead);
+      skip_other(ahead);
+    }
     uint32_t nt = 0;
     bool alive = true;
-    for (; wk.left > 0 && alive; wk.advance(a)) {
+    for (; wk.left > 0 && alive; wk.advance(a), ++nt) {
+      if ((nt & 1) != set) continue;  // the other set's tile
       const uint32_t sc = nt % SC, sa = nt % SA;
-      const long key = (long)(wk.r / a.Tq) * a.nc_max + (long)wk.j * kTcRows + t;
-      const bool in = wk.j * kTcRows + t < a.nc_max;
-      uint32_t sbytes = 0;  // the row's scale bytes (DI / 32 of them)
-      if (in) {
-        if constexpr (DI == 128) sbytes = __ldg(reinterpret_cast<const uint32_t *>(scales) + key);
-        else sbytes = __ldg(reinterpret_cast<const uint16_t *>(scales) + key);
-      }
+      const uint32_t sbytes = ring[0];
+#pragma unroll
+      for (int i = 0; i < kPre - 1; ++i) ring[i] = ring[i + 1];
+      ring[kPre - 1] = scale_word(ahead);
+      skip_other(ahead);
       bool ok = mbar_wait(c_full + 8 * sc, (nt / SC) & 1, abort);
       ok = ok && mbar_wait(a_empty + 8 * sa, ((nt / SA) & 1) ^ 1, abort);
       if (!__all_sync(0xffffffffu, ok)) {
@@ -373,7 +395,6 @@ __global__ void __launch_bounds__(kF4Threads, 1)
       fence_proxy_async_smem();  // the tile, visible to the tensor cores
       __syncwarp();
       if (lane == 0) mbar_arrive(a_full + 8 * sa);
-      ++nt;
     }
   }
 
