@@ -56,6 +56,7 @@ def _load():
         lib.orc_attend.argtypes = [P, P, P, I, P, P, P, I, I, I, I, I, I, I, I, D, P, I, P]
         lib.orc_quantize_mxfp4.argtypes = [P, I, L, I, P, P]
         lib.orc_dequant_mxfp4.argtypes = [P, P, L, I, P]
+        lib.orc_norm_rope.argtypes = [P, L, I, I, P, P, D, I, D, I, I, P]
         lib.orc_set_threads.argtypes = [I]
         lib.orc_get_threads.restype = I
         for name in ("orc_round", "orc_csa_compress", "orc_hca_compress", "orc_index_scores",
@@ -266,4 +267,26 @@ def dequant_mxfp4(codes, scales):
     rows = codes.size // (dI // 2)
     out = np.empty(codes.shape[:-1] + (dI,), np.float64)
     _check(lib.orc_dequant_mxfp4(pc, ps, rows, dI, out.ctypes.data_as(ctypes.c_void_p)), "dequant_mxfp4")
+    return out
+
+
+def norm_rope(x, pos, gamma=None, eps=1e-6, rope_dim=64, base=10000.0, norm=True, rotate=True,
+              inverse=False):
+    """QK-norm and partial RoPE of ``x`` ``[..., G, d]`` (the G heads of a
+    row share its position ``pos[...]``, shape ``x.shape[:-2]``): RMSNorm per
+    head with ``gamma`` ``[d]`` (ones when None), then a rotation of the last
+    ``rope_dim`` dims by ``+pos`` (``-pos`` when ``inverse``); the readings are
+    stated at ``orc_norm_rope``.  Returns float64 of the shape of ``x``."""
+    dt = _dt_of(x)
+    if gamma is not None:
+        _same_dt(x, gamma)
+    *lead, G, d = x.shape
+    R = int(np.prod(lead)) if lead else 1
+    p = np.ascontiguousarray(np.broadcast_to(np.asarray(pos, np.int64), tuple(lead)).reshape(R))
+    xc, px = _c(x)
+    gc, pg = (None, None) if gamma is None else _c(gamma)
+    out = np.empty(x.shape, np.float64)
+    flags = (1 if norm else 0) | (2 if rotate else 0) | (4 if inverse else 0)
+    _check(_load().orc_norm_rope(px, R, G, d, p.ctypes.data, pg, float(eps), int(rope_dim),
+                                 float(base), flags, dt, out.ctypes.data), "norm_rope")
     return out

@@ -574,3 +574,59 @@ int orc_dequant_mxfp4(const uint8_t *codes, const uint8_t *scales, long rows, in
     }
   return ORC_OK;
 }
+
+/* ------------------------------------------------------------------ */
+/* QK-norm and partial RoPE                                            */
+/* ------------------------------------------------------------------ */
+
+/*
+ * [A4] "The attention: compress, then select", third detail: queries and
+ * compressed entries are RMS-normalised per head, RoPE rotates only the last
+ * dims of each vector (64 of 512 there), and since the cached entry is also
+ * the value, each output is rotated back by its own query's position so that
+ * only relative position remains.  Readings (the pages give no formula):
+ *   RMSNorm  y[c] = x[c] / sqrt(mean_c(x^2) + eps) * gamma[c]  (gamma all
+ *            ones when NULL), over the d dims of one head;
+ *   RoPE     on the last r of the d dims, the adjacent pairs
+ *            (d-r+2j, d-r+2j+1), j = 0..r/2-1, rotated by the angle
+ *            p * base^(-2j/r):  (a, b) -> (a cos - b sin, a sin + b cos);
+ *            the textbook frequencies (base 10000 by default; the pages do
+ *            not mention the YaRN extension of the released model);
+ *   inverse  the same rotation by the angle -p.
+ * Normalisation comes first, then the rotation.
+ * x: [R][G][d] (G heads share the position pos[r]); gamma: [d] or NULL;
+ * flags: bit 0 normalise, bit 1 rotate, bit 2 rotate by -p instead of +p.
+ * out: [R][G][d] double, unrounded.
+ */
+int orc_norm_rope(const void *x, long R, int G, int d, const int64_t *pos, const void *gamma,
+                  double eps, int r, double base, int flags, int dt, double *out) {
+  if (!x || !pos || !out || R < 0 || G < 1 || d < 1 || r < 0 || r > d || (r & 1)) return ORC_ERR_ARG;
+  if (dt != ORC_F32 && dt != ORC_BF16) return ORC_ERR_ARG;
+  if ((flags & 1) && !(eps >= 0.0)) return ORC_ERR_ARG;
+  if ((flags & 2) && r > 0 && !(base > 0.0)) return ORC_ERR_ARG;
+#pragma omp parallel for schedule(static)
+  for (long row = 0; row < R * G; ++row) {
+    const long rr = row / G;
+    const size_t o = (size_t)row * d;
+    double *y = out + o;
+    for (int c = 0; c < d; ++c) y[c] = ld(x, dt, o + c);
+    if (flags & 1) {
+      double ss = 0.0;
+      for (int c = 0; c < d; ++c) ss += y[c] * y[c];
+      const double inv = 1.0 / sqrt(ss / d + eps);
+      for (int c = 0; c < d; ++c) y[c] = y[c] * inv * (gamma ? ld(gamma, dt, (size_t)c) : 1.0);
+    }
+    if ((flags & 2) && r > 0) {
+      const double p = (flags & 4) ? -(double)pos[rr] : (double)pos[rr];
+      for (int j = 0; j < r / 2; ++j) {
+        const double ang = p * pow(base, -2.0 * j / r);
+        const double cs = cos(ang), sn = sin(ang);
+        const int i0 = d - r + 2 * j, i1 = i0 + 1;
+        const double a = y[i0], b = y[i1];
+        y[i0] = a * cs - b * sn;
+        y[i1] = a * sn + b * cs;
+      }
+    }
+  }
+  return ORC_OK;
+}

@@ -1,7 +1,7 @@
 """Mutation check of the oracle's pins: each plausible mistake below (a
 swapped series, a transposed weight, a dropped ReLU or head weight, an
 off-by-one in visibility or the window, a wrong tie rule, a wrong scale,
-double rounding) is planted in a copy of the oracle's C source, compiled,
+double rounding, a wrong rotation or norm) is planted in a copy of the oracle's C source, compiled,
 and the pin tests are run against it.  Every mutant must fail at least one
 pin; a mutant that survives means the pins do not determine that part of
 the definition."""
@@ -17,7 +17,7 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 SRC = os.path.join(ROOT, "oracle", "csa_oracle.c")
 PINS = ["tests/test_oracle_compress.py", "tests/test_oracle_index_topk.py",
         "tests/test_oracle_attend.py", "tests/test_oracle_e2e.py",
-        "tests/test_oracle_mxfp4.py"]
+        "tests/test_oracle_mxfp4.py", "tests/test_oracle_rope.py"]
 
 MUTANTS = {
     "csa_series_swapped": ("const void *W = (j < 4) ? Wa : Wb;", "const void *W = (j < 4) ? Wb : Wa;"),
@@ -44,6 +44,12 @@ MUTANTS = {
     "attend_sink_ignored": ("if (sink) den += exp(sink[h] - mx);", ""),
     "mxfp4_ties_to_odd": ("return (lo % 2 == 0) ? lo : lo + 1;", "return (lo % 2 == 1) ? lo : lo + 1;"),
     "mxfp4_scale_off_by_one": ("X = ex - 1 - 2;", "X = ex - 1 - 1;"),
+    "rms_sum_not_mean": ("sqrt(ss / d + eps)", "sqrt(ss + eps)"),
+    "norm_gamma_ignored": ("y[c] * inv * (gamma ? ld(gamma, dt, (size_t)c) : 1.0)", "y[c] * inv"),
+    "rope_turns_backwards": ("const double cs = cos(ang), sn = sin(ang);", "const double cs = cos(ang), sn = -sin(ang);"),
+    "rope_half_split_pairs": ("const int i0 = d - r + 2 * j, i1 = i0 + 1;", "const int i0 = d - r + j, i1 = i0 + r / 2;"),
+    "rope_frequency_exponent": ("pow(base, -2.0 * j / r)", "pow(base, -1.0 * j / r)"),
+    "rope_inverse_ignored": ("(flags & 4) ? -(double)pos[rr] : (double)pos[rr]", "(double)pos[rr]"),
     "round_double_rounding": ("r = nearbyint(ldexp(a, -q));", "r = nearbyint(ldexp((double)(float)a, -q));"),
 }
 
