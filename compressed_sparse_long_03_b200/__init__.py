@@ -71,6 +71,9 @@ def lib() -> ctypes.CDLL:
         L.csa_topk.argtypes = [P, P, P, I, I, I, I, P, P]
         L.csa_attend.argtypes = [P, P, P, I, P, P, P, I, I, I, I, I, I, I, F, P, I, P, P]
         L.hca_attend.argtypes = [P, P, P, I, P, P, I, I, I, I, I, I, I, F, P, I, P, P]
+        L.csa_norm_rope.argtypes = [P, P, ctypes.c_long, I, I, P, P, I, I, I, P, F, I, F, I, I, P]
+        L.csa_attend_rope.argtypes = [P, P, P, I, P, P, P, I, I, I, I, I, I, I, F, P, P, F, I, F, I, I, P, P]
+        L.hca_attend_rope.argtypes = [P, P, P, I, P, P, I, I, I, I, I, I, I, F, P, P, F, I, F, I, I, P, P]
         for name in ("csa_check_device_error", "csa_compress", "hca_compress", "csa_compress_step",
                      "hca_compress_step", "csa_quantize_mxfp4", "csa_index_topk_mxfp4", "csa_index_topk",
                      "csa_index_topk_noalloc", "csa_index_scores", "csa_topk", "csa_attend", "hca_attend"):
@@ -321,4 +324,57 @@ def hca_attend(q, kv_c, kv_tok, lens, q_pos=None, m=128, window=128, scale=0.0, 
     _check(lib().hca_attend(_p(q), _p(kv_c), _p(kv_tok), kv_tok.shape[1], _i32(lens), _i32(q_pos),
                             B, Tq, H, d, kv_c.shape[1], m, window, float(scale), _f32(sink), _dt(q),
                             _p(out), _s(stream)))
+    return out
+
+
+# QK-norm and partial RoPE (csa_norm_rope flags)
+NR_NORM = 1
+NR_ROTATE = 2
+NR_INVERSE = 4
+
+
+def csa_norm_rope(x, y=None, pos=None, lens=None, Tq=1, pos_stride=1, pos_offset=0, gamma=None, eps=1e-6,
+                  rope_dim=64, rope_base=10000.0, flags=NR_NORM | NR_ROTATE, stream=None):
+    """x [R][G][d] (or [..., G, d]) -> y = RMSNorm and/or RoPE of every head
+    vector (in place when y is x); the position of row group r is pos[r],
+    else lens[r // Tq] - Tq + r % Tq, else pos_stride * (r % Tq) + pos_offset."""
+    *lead, G, d = x.shape
+    R = 1
+    for n in lead:
+        R *= n
+    if y is None:
+        y = torch.empty_like(x)
+    _check(lib().csa_norm_rope(_p(x), _p(y), R, G, d, _i32(pos), _i32(lens), int(Tq), int(pos_stride),
+                               int(pos_offset), _p(gamma), float(eps), int(rope_dim), float(rope_base),
+                               int(flags), _dt(x), _s(stream)))
+    return y
+
+
+def csa_attend_rope(q, kv_c, kv_tok, idx, lens, q_pos=None, window=128, scale=0.0, out=None, stream=None,
+                    sink=None, q_gamma=None, eps=1e-6, rope_dim=64, rope_base=10000.0,
+                    flags=NR_NORM | NR_ROTATE):
+    """csa_attend with the query's QK-norm / RoPE and the output's inverse
+    rotation fused into the attention kernel."""
+    B, Tq, H, d = q.shape
+    if out is None:
+        out = torch.empty_like(q)
+    _check(lib().csa_attend_rope(_p(q), _p(kv_c), _p(kv_tok), kv_tok.shape[1], _i32(idx), _i32(lens),
+                                 _i32(q_pos), B, Tq, H, d, kv_c.shape[1], idx.shape[-1], window, float(scale),
+                                 _f32(sink), _p(q_gamma), float(eps), int(rope_dim), float(rope_base),
+                                 int(flags), _dt(q), _p(out), _s(stream)))
+    return out
+
+
+def hca_attend_rope(q, kv_c, kv_tok, lens, q_pos=None, m=128, window=128, scale=0.0, out=None, stream=None,
+                    sink=None, q_gamma=None, eps=1e-6, rope_dim=64, rope_base=10000.0,
+                    flags=NR_NORM | NR_ROTATE):
+    """hca_attend with the query's QK-norm / RoPE and the output's inverse
+    rotation fused into the attention kernel."""
+    B, Tq, H, d = q.shape
+    if out is None:
+        out = torch.empty_like(q)
+    _check(lib().hca_attend_rope(_p(q), _p(kv_c), _p(kv_tok), kv_tok.shape[1], _i32(lens), _i32(q_pos),
+                                 B, Tq, H, d, kv_c.shape[1], m, window, float(scale), _f32(sink),
+                                 _p(q_gamma), float(eps), int(rope_dim), float(rope_base), int(flags), _dt(q),
+                                 _p(out), _s(stream)))
     return out

@@ -23,7 +23,10 @@
 
 #include <cooperative_groups.h>
 
+#include <type_traits>
+
 #include "common.cuh"
+#include "rope.cuh"
 
 namespace csa {
 
@@ -45,7 +48,25 @@ struct AttendArgs {
   const float *sink;  // [H] per-head sink logits (scaled-logit units), or nullptr
   int n_tok, k, Tq, H, nc_max, m, window;
   float scale_log2;  // softmax scale * log2(e)
+  // QK-norm and partial RoPE fused around the attention (third of the three
+  // details): qk_flags kNrNorm normalises each query head (q_gamma [d] or
+  // nullptr, q_eps), kNrRotate turns the query's last rope_r dims by its
+  // position t and the output's back by -t; 0: the query is used as given
+  int qk_flags, rope_r;
+  const void *q_gamma;
+  float q_eps;
+  double rope_log2_base;
 };
+
+// Round a float to the storage type T (what a staged query holds).
+template <typename T>
+__device__ __forceinline__ float round_as(float v) {
+  if constexpr (std::is_same<T, float>::value) {
+    return v;
+  } else {
+    return __bfloat162float(__float2bfloat16_rn(v));
+  }
+}
 
 // A head's sink logit in the kernels' base-2 units (-inf: no sink).  "Anatomy
 // of a Frontier Model", second of the three details: a learned per-head logit
@@ -75,6 +96,7 @@ __device__ __forceinline__ P *att_peer(P *mine, int rank) {
 template <typename T, int D, int CS>
 __global__ void __launch_bounds__(kAttThreads) k_attend_fma(AttendArgs a) {
   extern __shared__ float smem[];
+  __shared__ float2 rot_cs[64];  // (cos, sin) of the query position's RoPE angles
   const int H = a.H;
   float *qs = smem;                                   // [H][D]; later the partial outputs
   float *kt = qs + (size_t)H * D;                     // [kAttTile][D + 1]
@@ -126,6 +148,40 @@ __global__ void __launch_bounds__(kAttThreads) k_attend_fma(AttendArgs a) {
     load16(qrow + (size_t)u * V, f);
 #pragma unroll
     for (int j = 0; j < V; ++j) qs[u * V + j] = f[j];
+  }
+  if (a.qk_flags) {
+    // QK-norm and partial RoPE of the staged query heads, one warp per head,
+    // D / 32 consecutive dims per lane; the result is rounded to T as a
+    // normalised, rotated query stored in T would be
+    constexpr int E = D / 32;
+    if ((a.qk_flags & kNrRotate) && tid < a.rope_r / 2)
+      rot_cs[tid] = rope_cos_sin(t, rope_turns(tid, a.rope_r, a.rope_log2_base));
+    __syncthreads();
+    const int d0 = D - a.rope_r;
+    const T *gq = static_cast<const T *>(a.q_gamma);
+    for (int h = wid; h < H; h += kAttWarps) {
+      float x[E];
+#pragma unroll
+      for (int e = 0; e < E; ++e) x[e] = qs[(size_t)h * D + lane * E + e];
+      if (a.qk_flags & kNrNorm) {
+        float ss = 0.f;
+#pragma unroll
+        for (int e = 0; e < E; ++e) ss = fmaf(x[e], x[e], ss);
+        ss = warp_sum(ss);
+        const float inv = 1.f / sqrtf(ss / (float)D + a.q_eps);
+#pragma unroll
+        for (int e = 0; e < E; ++e) x[e] = x[e] * inv * (gq ? to_f(gq[lane * E + e]) : 1.f);
+      }
+      if (a.qk_flags & kNrRotate) {
+#pragma unroll
+        for (int e = 0; e < E; e += 2) {
+          const int i = lane * E + e;
+          if (i >= d0) rope_turn(x[e], x[e + 1], rot_cs[(i - d0) >> 1], false);
+        }
+      }
+#pragma unroll
+      for (int e = 0; e < E; ++e) qs[(size_t)h * D + lane * E + e] = round_as<T>(x[e]);
+    }
   }
 
   constexpr int EPL = D / 32;  // output elements per lane
@@ -225,7 +281,20 @@ __global__ void __launch_bounds__(kAttThreads) k_attend_fma(AttendArgs a) {
       Ls = fmaf(att_peer<CS>(pl, c)[h], wgt, Ls);
       Os = fmaf(att_peer<CS>(qs, c)[(size_t)h * D + e], wgt, Os);
     }
-    store_f(out + (size_t)h * D + e, Os / Ls);
+    float val = Os / Ls;
+    if (a.qk_flags & kNrRotate) {
+      // turn the output back by the query's position: the pair partner of
+      // dim e is dim e ^ 1, held by lane ^ 1 (D * nmine is a multiple of 64,
+      // so every lane of the warp is in this iteration)
+      const float other = __shfl_xor_sync(0xffffffffu, val, 1);
+      const int d0 = D - a.rope_r;
+      if (e >= d0) {
+        float u0 = (e & 1) ? other : val, u1 = (e & 1) ? val : other;
+        rope_turn(u0, u1, rot_cs[(e - d0) >> 1], true);
+        val = (e & 1) ? u1 : u0;
+      }
+    }
+    store_f(out + (size_t)h * D + e, val);
   }
   att_cluster_sync<CS>();  // peers may still be reading this CTA's partials
 }

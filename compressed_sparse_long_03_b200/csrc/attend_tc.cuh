@@ -62,6 +62,7 @@ __global__ void __launch_bounds__(kAtThreads, 1) k_attend_tc(AttendArgs a) {
   __shared__ float xmax[2][128];       // per-half row max (then sum) of the partner
   __shared__ float mw[136], minv[128];  // merge weights [hl * CS + c], 1 / sum
   __shared__ int abort_flag;
+  __shared__ float2 rot_cs[64];  // (cos, sin) of the query position's RoPE angles
 
   uint8_t *base = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -135,6 +136,8 @@ __global__ void __launch_bounds__(kAtThreads, 1) k_attend_tc(AttendArgs a) {
   const int L = nsel + nwin;
   const int per = (L + CS - 1) / CS;
   const int lo = min(L, rank * per), hi = min(L, lo + per);
+  if ((a.qk_flags & kNrRotate) && tid < a.rope_r / 2)
+    rot_cs[tid] = rope_cos_sin(t, rope_turns(tid, a.rope_r, a.rope_log2_base));
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -217,6 +220,63 @@ __global__ void __launch_bounds__(kAtThreads, 1) k_attend_tc(AttendArgs a) {
     tc_fence_after();
     if constexpr (NKB == 2) {
       if (pn < hi) gather(pn, kb ^ 1);  // the next tile's rows during this tile's math
+    }
+    if (a.qk_flags && p0 == lo) {
+      // QK-norm and partial RoPE of the staged query rows, in place, before
+      // the first S = Q K^T: this thread's 64 columns of head hrow are the 8
+      // swizzled 16-byte chunks of row hrow in Q atom `half`; the row's sum
+      // of squares is completed through the partner thread
+      const uint32_t qa = smem_u32(sQ) + half * kAtQAtom + hrow * 128;
+      float ss = 0.f;
+      if (hrow < H) {
+#pragma unroll
+        for (int cc = 0; cc < 8; ++cc) {
+          uint32_t w0_, w1_, w2_, w3_;
+          asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                       : "=r"(w0_), "=r"(w1_), "=r"(w2_), "=r"(w3_)
+                       : "r"(qa + ((cc ^ (hrow & 7)) << 4)));
+          const uint32_t w[4] = {w0_, w1_, w2_, w3_};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float x0 = __uint_as_float(w[e] << 16), x1 = __uint_as_float(w[e] & 0xFFFF0000u);
+            ss = fmaf(x0, x0, fmaf(x1, x1, ss));
+          }
+        }
+      }
+      xmax[half][hrow] = ss;
+      __syncthreads();
+      ss += xmax[half ^ 1][hrow];
+      const float inv = (a.qk_flags & kNrNorm) ? 1.f / sqrtf(ss / (float)D + a.q_eps) : 1.f;
+      const int d0 = D - a.rope_r;
+      const __nv_bfloat16 *gq = (a.qk_flags & kNrNorm) ? static_cast<const __nv_bfloat16 *>(a.q_gamma) : nullptr;
+      if (hrow < H) {
+#pragma unroll
+        for (int cc = 0; cc < 8; ++cc) {
+          const uint32_t addr = qa + ((cc ^ (hrow & 7)) << 4);
+          uint32_t w0_, w1_, w2_, w3_;
+          asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                       : "=r"(w0_), "=r"(w1_), "=r"(w2_), "=r"(w3_)
+                       : "r"(addr));
+          uint32_t w[4] = {w0_, w1_, w2_, w3_};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int col = half * (D / 2) + cc * 8 + 2 * e;
+            float x0 = __uint_as_float(w[e] << 16) * inv, x1 = __uint_as_float(w[e] & 0xFFFF0000u) * inv;
+            if (gq) {
+              x0 *= __bfloat162float(gq[col]);
+              x1 *= __bfloat162float(gq[col + 1]);
+            }
+            if ((a.qk_flags & kNrRotate) && col >= d0) rope_turn(x0, x1, rot_cs[(col - d0) >> 1], false);
+            __nv_bfloat162 pr = __floats2bfloat162_rn(x0, x1);
+            w[e] = *reinterpret_cast<uint32_t *>(&pr);
+          }
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(w[0]), "r"(w[1]), "r"(w[2]),
+                       "r"(w[3])
+                       : "memory");
+        }
+      }
+      fence_proxy_async_smem();
+      __syncthreads();
     }
     const uint32_t sKb = smem_u32(sK) + kb * 2 * kAtKHalf;
     // ---- S = Q K^T
@@ -354,7 +414,11 @@ __global__ void __launch_bounds__(kAtThreads, 1) k_attend_tc(AttendArgs a) {
         uint32_t w4[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          __nv_bfloat162 pr = __floats2bfloat162_rn(o[8 * j + 2 * e] * f, o[8 * j + 2 * e + 1] * f);
+          float x0 = o[8 * j + 2 * e] * f, x1 = o[8 * j + 2 * e + 1] * f;
+          const int col = half * (D / 2) + 8 * j + 2 * e;
+          if ((a.qk_flags & kNrRotate) && col >= D - a.rope_r)  // back by the query's position
+            rope_turn(x0, x1, rot_cs[(col - (D - a.rope_r)) >> 1], true);
+          __nv_bfloat162 pr = __floats2bfloat162_rn(x0, x1);
           w4[e] = *reinterpret_cast<uint32_t *>(&pr);
         }
         dst[j] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
@@ -409,8 +473,17 @@ __global__ void __launch_bounds__(kAtThreads, 1) k_attend_tc(AttendArgs a) {
       acc.w = fmaf(p.w, wgt, acc.w);
     }
     const float il = minv[hl];
-    __nv_bfloat162 lo2 = __floats2bfloat162_rn(acc.x * il, acc.y * il);
-    __nv_bfloat162 hi2 = __floats2bfloat162_rn(acc.z * il, acc.w * il);
+    acc.x *= il;
+    acc.y *= il;
+    acc.z *= il;
+    acc.w *= il;
+    if (a.qk_flags & kNrRotate) {  // back by the query's position
+      const int d0 = D - a.rope_r;
+      if (4 * j >= d0) rope_turn(acc.x, acc.y, rot_cs[(4 * j - d0) >> 1], true);
+      if (4 * j + 2 >= d0) rope_turn(acc.z, acc.w, rot_cs[(4 * j + 2 - d0) >> 1], true);
+    }
+    __nv_bfloat162 lo2 = __floats2bfloat162_rn(acc.x, acc.y);
+    __nv_bfloat162 hi2 = __floats2bfloat162_rn(acc.z, acc.w);
     uint2 pk;
     pk.x = *reinterpret_cast<uint32_t *>(&lo2);
     pk.y = *reinterpret_cast<uint32_t *>(&hi2);

@@ -7,6 +7,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <cmath>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
@@ -29,6 +30,7 @@
 #include "topk.cuh"
 #include "attend_fma.cuh"
 #include "attend_tc.cuh"
+#include "rope.cuh"
 
 namespace {
 
@@ -580,12 +582,46 @@ int launch_attend_tc(const csa::AttendArgs &a, int R, cudaStream_t st, const cha
   return launch_cluster(kern, cs, (unsigned)cs * R, csa::kAtThreads, smem, st, what, a);
 }
 
+// QK-norm / partial RoPE arguments of the fused attention entry points.
+struct QkSpec {
+  int flags = 0;  // CSA_NR_NORM | CSA_NR_ROTATE, 0: none
+  const void *gamma = nullptr;
+  float eps = 0.f;
+  int rope_dim = 0;
+  float rope_base = 0.f;
+};
+
+// Validation shared by csa_norm_rope and the fused attention.
+int check_norm_rope(const char *what, int d, int flags, float eps, int rope_dim, float rope_base,
+                    const void *gamma) {
+  if (flags & ~(CSA_NR_NORM | CSA_NR_ROTATE | CSA_NR_INVERSE))
+    return fail(CSA_ERR_UNSUPPORTED, "%s: unknown flags 0x%x", what, flags);
+  if ((flags & CSA_NR_NORM) && !(eps >= 0.f && eps < INFINITY))
+    return fail(CSA_ERR_SHAPE, "%s: eps must be finite and >= 0", what);
+  if (flags & CSA_NR_ROTATE) {
+    if (rope_dim < 0 || rope_dim > d || (rope_dim & 1))
+      return fail(CSA_ERR_UNSUPPORTED, "%s: rope_dim=%d must be even and in [0, d=%d]", what, rope_dim, d);
+    if (!(rope_base > 0.f && rope_base < INFINITY))
+      return fail(CSA_ERR_SHAPE, "%s: rope_base must be finite and > 0", what);
+  }
+  if (gamma && (reinterpret_cast<uintptr_t>(gamma) & 3))
+    return fail(CSA_ERR_ALIGN, "%s: gamma must be 4-byte aligned", what);
+  return CSA_OK;
+}
+
 int attend_common(const void *q, const void *kv_c, const void *kv_tok, int n_tok,
                   const int32_t *idx, const int32_t *lens, const int32_t *q_pos, int B, int Tq,
                   int H, int d, int nc_max, int k, int m, int window, float scale,
-                  const float *sink, csa_dtype dt, void *out, void *stream, const char *what) {
+                  const float *sink, csa_dtype dt, void *out, void *stream, const char *what,
+                  const QkSpec &qk = QkSpec()) {
   int rc = check_dtype(dt, what);
   if (rc) return rc;
+  if (qk.flags) {
+    if (qk.flags & CSA_NR_INVERSE)
+      return fail(CSA_ERR_UNSUPPORTED, "%s: the output's inverse rotation follows CSA_NR_ROTATE", what);
+    rc = check_norm_rope(what, d, qk.flags, qk.eps, qk.rope_dim, qk.rope_base, qk.gamma);
+    if (rc) return rc;
+  }
   if (B < 0 || Tq < 0) return fail(CSA_ERR_SHAPE, "%s: B=%d and Tq=%d must be >= 0", what, B, Tq);
   if ((long)B * Tq == 0) return CSA_OK;
   if (!q || !kv_tok || !lens || !out || (idx == nullptr && k > 0) || (nc_max > 0 && !kv_c))
@@ -617,6 +653,11 @@ int attend_common(const void *q, const void *kv_c, const void *kv_tok, int n_tok
   a.window = window;
   const float sc = scale > 0.f ? scale : 1.0f / sqrtf((float)d);
   a.scale_log2 = sc * 1.4426950408889634f;
+  a.qk_flags = qk.flags;
+  a.rope_r = (qk.flags & CSA_NR_ROTATE) ? qk.rope_dim : 0;
+  a.q_gamma = (qk.flags & CSA_NR_NORM) ? qk.gamma : nullptr;
+  a.q_eps = qk.eps;
+  a.rope_log2_base = (qk.flags & CSA_NR_ROTATE) ? std::log2((double)qk.rope_base) : 0.0;
   const int R = B * Tq;
   const long max_keys = (idx ? (long)k : (long)nc_max) + window;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -899,6 +940,84 @@ int hca_attend(const void *q, const void *kv_c, const void *kv_tok, int n_tok,
   if (nc_max > 65536) return fail(CSA_ERR_UNSUPPORTED, "hca_attend: nc_max=%d > 65536", nc_max);
   return attend_common(q, kv_c, kv_tok, n_tok, nullptr, lens, q_pos, B, Tq, H, d, nc_max, 0, m,
                        window, scale, sink, dt, out, stream, "hca_attend");
+}
+
+int csa_norm_rope(const void *x, void *y, long R, int G, int d, const int32_t *pos, const int32_t *lens,
+                  int Tq, int pos_stride, int pos_offset, const void *gamma, float eps, int rope_dim,
+                  float rope_base, int flags, csa_dtype dt, void *stream) {
+  const char *what = "csa_norm_rope";
+  begin_call();
+  int rc = check_dtype(dt, what);
+  if (rc) return rc;
+  if (d != 64 && d != 128) return fail(CSA_ERR_UNSUPPORTED, "%s: d=%d not in {64,128}", what, d);
+  if (R < 0 || G < 1) return fail(CSA_ERR_SHAPE, "%s: R=%ld must be >= 0 and G=%d >= 1", what, R, G);
+  if ((flags & CSA_NR_INVERSE) && !(flags & CSA_NR_ROTATE))
+    return fail(CSA_ERR_UNSUPPORTED, "%s: CSA_NR_INVERSE needs CSA_NR_ROTATE", what);
+  rc = check_norm_rope(what, d, flags, eps, rope_dim, rope_base, gamma);
+  if (rc) return rc;
+  if (!pos && Tq < 1) return fail(CSA_ERR_SHAPE, "%s: Tq=%d must be >= 1 without pos", what, Tq);
+  if (R == 0) return CSA_OK;
+  if (!x || !y) return fail(CSA_ERR_NULL, "%s: x and y must not be NULL", what);
+  if (!aligned16(x) || !aligned16(y)) return fail(CSA_ERR_ALIGN, "%s: x and y must be 16-byte aligned", what);
+  const long rows = R * (long)G;
+  if (rows / G != R || rows > (1L << 40)) return fail(CSA_ERR_UNSUPPORTED, "%s: too many rows", what);
+  csa::NormRopeArgs a;
+  a.x = x;
+  a.y = y;
+  a.rows = rows;
+  a.G = G;
+  a.pos = pos;
+  a.lens = pos ? nullptr : lens;
+  a.Tq = Tq < 1 ? 1 : Tq;
+  a.stride = pos_stride;
+  a.offset = pos_offset;
+  a.gamma = (flags & CSA_NR_NORM) ? gamma : nullptr;
+  a.eps = eps;
+  a.r = (flags & CSA_NR_ROTATE) ? rope_dim : 0;
+  a.flags = flags;
+  a.log2_base = (flags & CSA_NR_ROTATE) ? std::log2((double)rope_base) : 0.0;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const long want = (rows + 8 * csa::kNrUnroll - 1) / (8 * csa::kNrUnroll);  // 8 warps per CTA
+  const unsigned grid = (unsigned)std::max(1L, std::min(want, 8L * num_sms()));  // one wave
+  if (dt == CSA_F32)
+    return d == 64 ? launch_cluster(csa::k_norm_rope<float, 64>, 1, grid, csa::kNrThreads, 0, st, what, a)
+                   : launch_cluster(csa::k_norm_rope<float, 128>, 1, grid, csa::kNrThreads, 0, st, what, a);
+  return d == 64 ? launch_cluster(csa::k_norm_rope<__nv_bfloat16, 64>, 1, grid, csa::kNrThreads, 0, st, what, a)
+                 : launch_cluster(csa::k_norm_rope<__nv_bfloat16, 128>, 1, grid, csa::kNrThreads, 0, st, what, a);
+}
+
+int csa_attend_rope(const void *q, const void *kv_c, const void *kv_tok, int n_tok, const int32_t *idx,
+                    const int32_t *lens, const int32_t *q_pos, int B, int Tq, int H, int d, int nc_max,
+                    int k, int window, float scale, const float *sink, const void *q_gamma, float eps,
+                    int rope_dim, float rope_base, int flags, csa_dtype dt, void *out, void *stream) {
+  begin_call();
+  if (k < 1 || k > 4096) return fail(CSA_ERR_UNSUPPORTED, "csa_attend_rope: k=%d not in [1,4096]", k);
+  if (!idx && (long)B * Tq > 0) return fail(CSA_ERR_NULL, "csa_attend_rope: idx is NULL");
+  QkSpec qk;
+  qk.flags = flags;
+  qk.gamma = q_gamma;
+  qk.eps = eps;
+  qk.rope_dim = rope_dim;
+  qk.rope_base = rope_base;
+  return attend_common(q, kv_c, kv_tok, n_tok, idx, lens, q_pos, B, Tq, H, d, nc_max, k, 4, window,
+                       scale, sink, dt, out, stream, "csa_attend_rope", qk);
+}
+
+int hca_attend_rope(const void *q, const void *kv_c, const void *kv_tok, int n_tok,
+                    const int32_t *lens, const int32_t *q_pos, int B, int Tq, int H, int d, int nc_max,
+                    int m, int window, float scale, const float *sink, const void *q_gamma, float eps,
+                    int rope_dim, float rope_base, int flags, csa_dtype dt, void *out, void *stream) {
+  begin_call();
+  if (m < 1 || m > 4096) return fail(CSA_ERR_UNSUPPORTED, "hca_attend_rope: m=%d not in [1,4096]", m);
+  if (nc_max > 65536) return fail(CSA_ERR_UNSUPPORTED, "hca_attend_rope: nc_max=%d > 65536", nc_max);
+  QkSpec qk;
+  qk.flags = flags;
+  qk.gamma = q_gamma;
+  qk.eps = eps;
+  qk.rope_dim = rope_dim;
+  qk.rope_base = rope_base;
+  return attend_common(q, kv_c, kv_tok, n_tok, nullptr, lens, q_pos, B, Tq, H, d, nc_max, 0, m,
+                       window, scale, sink, dt, out, stream, "hca_attend_rope", qk);
 }
 
 }  // extern "C"

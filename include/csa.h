@@ -322,6 +322,70 @@ CSA_API int hca_attend(const void *q, const void *kv_c, const void *kv_tok, int 
                int m, int window, float scale, const float *sink, csa_dtype dt, void *out,
                void *stream);
 
+/* ------------------------------------------------------------------------
+ * QK-norm and partial RoPE.
+ *
+ * Anatomy page, "The attention: compress, then select", third of the three
+ * details: queries and compressed entries are RMS-normalised per head, RoPE
+ * turns only the last dims of each vector (64 of 512 there), and because
+ * the cached entry is also the value, each attention output is turned back
+ * by its own query's position, leaving only relative position.  Reading
+ * (the pages give no formula), per head vector of d dims:
+ *   CSA_NR_NORM    y = x / sqrt(mean(x^2) + eps) * gamma (gamma [d] in dt,
+ *                  or NULL for ones)
+ *   CSA_NR_ROTATE  after the norm, the adjacent pairs (d-r+2j, d-r+2j+1)
+ *                  of the last r = rope_dim dims turned by the angle
+ *                  p * rope_base^(-2j/r):  (a, b) -> (a cos - b sin,
+ *                  a sin + b cos)   (textbook RoPE frequencies)
+ *   CSA_NR_INVERSE with CSA_NR_ROTATE: the angle -p (undoes the rotation)
+ * Positions: a query at t (the attention's decode rule), a window token at
+ * its own position s, compressed entry i of stride m at m * i (the first
+ * token of its own block).
+ * ---------------------------------------------------------------------- */
+#define CSA_NR_NORM 1
+#define CSA_NR_ROTATE 2
+#define CSA_NR_INVERSE 4
+
+/* csa_norm_rope -- y = the flags' steps applied to x, per head vector.
+ *   x, y   [R][G][d] in dt (y may be x: in place; 16-byte aligned)
+ *   G      heads sharing one position (H for queries, 1 for caches)
+ *   position of row group r, first rule that applies:
+ *     pos    [R] int32 (explicit positions), else
+ *     lens   [R / Tq] int32: lens[r / Tq] - Tq + r % Tq (decode queries:
+ *            the attention's rule for q_pos == NULL), else
+ *     pos_stride * (r % Tq) + pos_offset  (a cache [B][Tq = nc_max][d] of
+ *            stride m: pos_stride = m; a token array [B][Tq = n][d]:
+ *            pos_stride = 1)
+ *   eps    >= 0; rope_dim even, 0 <= rope_dim <= d; rope_base > 0
+ * Supported: d in {64, 128}.  Caller owns every buffer; nothing is
+ * allocated; asynchronous on `stream`.
+ * ---------------------------------------------------------------------- */
+CSA_API int csa_norm_rope(const void *x, void *y, long R, int G, int d, const int32_t *pos,
+                          const int32_t *lens, int Tq, int pos_stride, int pos_offset, const void *gamma,
+                          float eps, int rope_dim, float rope_base, int flags, csa_dtype dt, void *stream);
+
+/* csa_attend_rope / hca_attend_rope -- csa_attend / hca_attend with the
+ * query's QK-norm and RoPE and the output's inverse rotation fused into the
+ * attention kernel:
+ *   q' = csa_norm_rope(q) at the query's position t with `flags`
+ *        (CSA_NR_NORM and/or CSA_NR_ROTATE; q_gamma, eps, rope_dim,
+ *        rope_base as there), rounded to dt as a stored q' would be;
+ *   o  = the attention of q' over the entries and window tokens, which the
+ *        caller has normalised and rotated at their own positions (e.g. by
+ *        csa_norm_rope when they are formed);
+ *   out = o turned back by -t when CSA_NR_ROTATE is set.
+ * Other arguments, supported sets and errors as csa_attend / hca_attend;
+ * CSA_NR_INVERSE is rejected (CSA_ERR_UNSUPPORTED).
+ * ---------------------------------------------------------------------- */
+CSA_API int csa_attend_rope(const void *q, const void *kv_c, const void *kv_tok, int n_tok, const int32_t *idx,
+                            const int32_t *lens, const int32_t *q_pos, int B, int Tq, int H, int d, int nc_max,
+                            int k, int window, float scale, const float *sink, const void *q_gamma, float eps,
+                            int rope_dim, float rope_base, int flags, csa_dtype dt, void *out, void *stream);
+CSA_API int hca_attend_rope(const void *q, const void *kv_c, const void *kv_tok, int n_tok,
+                            const int32_t *lens, const int32_t *q_pos, int B, int Tq, int H, int d, int nc_max,
+                            int m, int window, float scale, const float *sink, const void *q_gamma, float eps,
+                            int rope_dim, float rope_base, int flags, csa_dtype dt, void *out, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

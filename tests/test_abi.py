@@ -127,3 +127,35 @@ def test_binding_refuses_cpu_tensors(L):
     with pytest.raises(ValueError):
         csa.csa_compress(x, torch.zeros(1, dtype=torch.int32), torch.zeros(64, 64),
                          torch.zeros(64, 64), torch.zeros(8, 64))
+
+
+def nr_call(L, **kw):
+    a = dict(x=A16, y=A16, R=4, G=1, d=128, pos=None, lens=None, Tq=1, stride=1, offset=0, gamma=None,
+             eps=1e-6, rope_dim=64, base=10000.0, flags=3, dt=1)
+    a.update(kw)
+    return L.csa_norm_rope(a["x"], a["y"], a["R"], a["G"], a["d"], a["pos"], a["lens"], a["Tq"], a["stride"],
+                           a["offset"], a["gamma"], ctypes.c_float(a["eps"]), a["rope_dim"],
+                           ctypes.c_float(a["base"]), a["flags"], a["dt"], None)
+
+
+def test_norm_rope_validation(L):
+    assert nr_call(L, d=96) == E_UNSUP
+    assert nr_call(L, rope_dim=63) == E_UNSUP
+    assert nr_call(L, rope_dim=130) == E_UNSUP
+    assert nr_call(L, flags=8) == E_UNSUP
+    assert nr_call(L, flags=4) == E_UNSUP          # inverse without rotation
+    assert nr_call(L, eps=-1.0) == E_SHAPE
+    assert nr_call(L, base=0.0) == E_SHAPE
+    assert nr_call(L, G=0) == E_SHAPE
+    assert nr_call(L, Tq=0) == E_SHAPE
+    assert nr_call(L, x=None) == E_NULL
+    assert nr_call(L, y=A4) == E_ALIGN
+    assert nr_call(L, dt=3) == E_DTYPE
+    assert nr_call(L, R=0) == OK
+    # the fused attention refuses the inverse flag (the output's turn back follows the rotation)
+    rc = L.csa_attend_rope(A16, A16, A16, 128, A16, A16, None, 1, 1, 4, 128, 8, 4, 128, ctypes.c_float(0.0),
+                           None, None, ctypes.c_float(1e-6), 64, ctypes.c_float(1e4), 6, 1, A16, None)
+    assert rc == E_UNSUP
+    rc = L.hca_attend_rope(A16, A16, A16, 128, A16, None, 1, 1, 4, 128, 8, 128, 128, ctypes.c_float(0.0),
+                           None, None, ctypes.c_float(1e-6), 63, ctypes.c_float(1e4), 2, 1, A16, None)
+    assert rc == E_UNSUP

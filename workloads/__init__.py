@@ -56,6 +56,7 @@ _STREAMS = {
     "kI": 12, "kv": 13, "win": 14,
     "hca_kv": 15, "hca_W": 16, "hca_beta": 17, "hca_x": 18, "q2": 19,
     "lens": 20, "needle_pos": 21,
+    "q_gamma": 22, "kv_gamma": 23,
 }
 
 HERE = os.path.dirname(os.path.abspath(__file__))
