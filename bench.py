@@ -46,10 +46,11 @@ def parse():
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-steps", type=int, default=1, help="oracle steps for cpu_baseline")
-    p.add_argument("--workload", type=int, default=4, choices=[1, 2, 3, 4, 5, 6],
+    p.add_argument("--workload", type=int, default=4, choices=[1, 2, 3, 4, 5, 6, 7],
                    help="4 (default): the 1M CSA decode step; 1, 2, 3, 5: the other "
                         "workloads, one measurement line each (single GPU); 6: workload 4 "
-                        "with its indexer keys in MXFP4")
+                        "with its indexer keys in MXFP4; 7: workload 4 with QK-norm and "
+                        "partial RoPE")
     return p.parse_args()
 
 
@@ -397,6 +398,38 @@ def other_workload_plan(wid, wl, csa, torch, D):
         flops = B * (2.0 * nc * HI * dI + 4.0 * (k + window) * H * d)
         return stages, "queries/s", B, byts, flops, ("one decode step of the 1M workload with the indexer "
                                                       "keys in MXFP4 (68 B per key): indexer + top-k, attention")
+    if wid == 7:
+        B, nc, H, d, dI, HI = s["B"], s["nc"], s["H"], s["d"], s["dI"], s["HI"]
+        n_tok = D["win"].shape[1]
+        # the caches as the decode step keeps them: entries normalised and
+        # rotated when formed (entry i at 4 i), window tokens at their positions
+        D["q_gamma"] = to_dev_like(torch, W.normal(W.seed_of(4), "q_gamma", (d,), 1.0, "bf16"))
+        D["kv_gamma"] = to_dev_like(torch, W.normal(W.seed_of(4), "kv_gamma", (d,), 1.0, "bf16"))
+        D["kv_r"] = torch.empty_like(D["kv"])
+        csa.csa_norm_rope(D["kv"].view(B, nc, 1, d), D["kv_r"].view(B, nc, 1, d), gamma=D["kv_gamma"], Tq=nc,
+                          pos_stride=4, flags=3)
+        lens = wl["lens"].astype(np.int64)
+        j = np.arange(n_tok)[None, :]
+        ring_pos = np.where(lens[:, None] - 1 >= j, j + n_tok * ((lens[:, None] - 1 - j) // n_tok), 0)
+        D["win_r"] = csa.csa_norm_rope(D["win"].view(B, n_tok, 1, d), gamma=D["kv_gamma"],
+                                       pos=to_dev_i32(torch, ring_pos.astype(np.int32)),
+                                       flags=3).view(B, n_tok, d)
+        torch.cuda.synchronize()
+        idx = torch.empty(B, 1, k, dtype=torch.int32, device="cuda")
+        out = torch.empty(B, 1, H, d, dtype=torch.bfloat16, device="cuda")
+        ws = csa.index_topk_workspace(B, 1, nc, False)
+        stages = [
+            ("csa_index_topk", lambda: csa.csa_index_topk(D["qI"], D["w"], D["kI"], D["lens"], k,
+                                                          idx_out=idx, workspace=ws)),
+            ("csa_attend_rope", lambda: csa.csa_attend_rope(D["q"], D["kv_r"], D["win_r"], idx, D["lens"],
+                                                            window=window, out=out, q_gamma=D["q_gamma"])),
+        ]
+        byts = B * (nc * dI * 2 + (k + window) * d * 2 + (2 * H * d + HI * dI + HI) * 2) + d * 2
+        flops = B * (2.0 * nc * HI * dI + 4.0 * (k + window) * H * d)
+        return stages, "queries/s", B, byts, flops, ("one decode step of the 1M workload with QK-norm and "
+                                                      "partial RoPE: indexer + top-k, attention with the "
+                                                      "query's norm / rotation and the output's inverse "
+                                                      "rotation fused in")
     if wid == 5:
         B, H, d, dI, HI, m = s["B"], s["H"], s["d"], s["dI"], s["HI"], s["m"]
         nc = s["nc"]
@@ -431,7 +464,7 @@ def run_other_workload(args):
     from tests.helpers import to_dev
     torch.cuda.set_device(0)
     wid = args.workload
-    wl = W.make(4 if wid == 6 else wid)
+    wl = W.make(4 if wid in (6, 7) else wid)
     D = {n: to_dev(wl[n]) for n in wl.arrays if n != "needle_pos"}
     stages, unit, units, byts, flops, what = other_workload_plan(wid, wl, csa, torch, D)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
@@ -485,7 +518,7 @@ def run_other_workload(args):
     tfl = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     gbs = byts / (ms * 1e-3) / 1e9
     tfs = flops / (ms * 1e-3) / 1e12
-    name = "csa_decode_mxfp4keys_b4_n1048576" if wid == 6 else wl.name
+    name = {6: "csa_decode_mxfp4keys_b4_n1048576", 7: "csa_decode_qknorm_rope_b4_n1048576"}.get(wid, wl.name)
     line = {"metric": f"{name}: {unit}", "value": units * 1000.0 / ms, "unit": unit, "n_gpus": 1,
             "steps": K, "warmup": max(3, args.warmup), "ms_per_step": ms, "higher_is_better": True,
             "dtype": wl.dt, "data": "synthetic (seeded PCG64)",
@@ -501,6 +534,8 @@ def run_other_workload(args):
         line["hca_compress"] = time_hca_compress(wl, csa, torch, flush, min(K, 20), hbm)
     if wid == 5:
         line["compress_step"] = time_compress_step(wl, csa, torch, D, flush, min(K, 20))
+    if wid == 7:
+        line["norm_rope_cache"] = time_norm_rope_cache(wl, csa, torch, D, min(K, 50), hbm)
     if not args.no_cpu_baseline:
         line["cpu_baseline"] = oracle_sample(wid, wl)
     print(json.dumps(line))
@@ -554,6 +589,32 @@ def oracle_sample(wid, wl):
         t = clock(one)
         return {"value": 1.0 / t, "unit": "queries/s", "cores": cores, "kind": "oracle",
                 "sample": "one query of the batch (its keys quantised, dequantised, scored; attention)"}
+    if wid == 7:
+        sl = slice(0, 1)
+        d, nc = s["d"], s["nc"]
+        gq = W.normal(W.seed_of(4), "q_gamma", (d,), 1.0, "bf16")
+        gk = W.normal(W.seed_of(4), "kv_gamma", (d,), 1.0, "bf16")
+        lens = wl["lens"][sl].astype(np.int64)
+        n_tok = wl["win"].shape[1]
+
+        # the caches as the step finds them (normalised and rotated when formed)
+        kv_r = oracle.round_to(oracle.norm_rope(wl["kv"][sl][:, :, None, :], 4 * np.arange(nc)[None, :],
+                                                gamma=gk)[:, :, 0, :], oracle.BF16)
+        j = np.arange(n_tok)[None, :]
+        rp = np.where(lens[:, None] - 1 >= j, j + n_tok * ((lens[:, None] - 1 - j) // n_tok), 0)
+        win_r = oracle.round_to(oracle.norm_rope(wl["win"][sl][:, :, None, :], rp, gamma=gk)[:, :, 0, :],
+                                oracle.BF16)
+
+        def one():
+            t = (lens - 1)[:, None]
+            idx, _ = oracle.index_topk(wl["qI"][sl], wl["w"][sl], wl["kI"][sl], wl["lens"][sl], k)
+            q_r = oracle.round_to(oracle.norm_rope(wl["q"][sl], t, gamma=gq), oracle.BF16)
+            o = oracle.attend(q_r, kv_r, win_r, wl["lens"][sl], idx=idx, window=window)
+            oracle.norm_rope(o.astype(np.float32), t, norm=False, inverse=True)
+        t = clock(one)
+        return {"value": 1.0 / t, "unit": "queries/s", "cores": cores, "kind": "oracle",
+                "sample": "one query of the batch (indexer + top-k, the query normalised and rotated, "
+                          "attention, the output turned back)"}
     if wid == 3:
         nq = 4
         sl = slice(0, nq)
@@ -621,6 +682,35 @@ def time_compress_step(wl, csa, torch, D, flush, K):
             "calls": "csa_compress_step (KV) + csa_compress_step (indexer keys) + hca_compress_step",
             "timing": "sum of the three kernels' device times",
             "note": "every sequence completes a CSA and an HCA block in this step"}
+
+
+def to_dev_like(torch, a):
+    """numpy float32 / bf16 bits (uint16) -> CUDA tensor."""
+    from tests.helpers import to_dev
+    return to_dev(a)
+
+
+def time_norm_rope_cache(wl, csa, torch, D, K, hbm):
+    """csa_norm_rope over the whole 1M-token entry cache (B x 262,144 entries
+    of 256 B: read once, written once; 512 MiB per launch, larger than L2)."""
+    s = wl.sizes
+    B, nc, d = s["B"], s["nc"], s["d"]
+    src, dst = D["kv"].view(B, nc, 1, d), D["kv_r"].view(B, nc, 1, d)
+    for _ in range(3):
+        csa.csa_norm_rope(src, dst, gamma=D["kv_gamma"], Tq=nc, pos_stride=4, flags=3)
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    for a, b in ev:
+        a.record()
+        csa.csa_norm_rope(src, dst, gamma=D["kv_gamma"], Tq=nc, pos_stride=4, flags=3)
+        b.record()
+    torch.cuda.synchronize()
+    csa.check_device_error()
+    us = 1000 * statistics.median(a.elapsed_time(b) for a, b in ev)
+    byts = 2 * B * nc * d * 2
+    gbs = byts / (us * 1e-6) / 1e9
+    return {"kernel": "k_norm_rope<bf16,128>", "rows": B * nc, "us": us, "bytes_per_launch": byts,
+            "achieved_gbs": gbs, "frac_of_measured_hbm": gbs / hbm, "bound": "hbm"}
 
 
 def to_dev_i32(torch, a):

@@ -63,6 +63,7 @@ __global__ void __launch_bounds__(kAtThreads, 1) k_attend_tc(AttendArgs a) {
   __shared__ float mw[136], minv[128];  // merge weights [hl * CS + c], 1 / sum
   __shared__ int abort_flag;
   __shared__ float2 rot_cs[64];  // (cos, sin) of the query position's RoPE angles
+  __shared__ float sgam[128];    // the query's RMSNorm gain (QK-norm)
 
   uint8_t *base = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -104,6 +105,9 @@ __global__ void __launch_bounds__(kAtThreads, 1) k_attend_tc(AttendArgs a) {
     const uint32_t dst = smem_u32(sQ) + (c >> 3) * kAtQAtom + h * 128 + (((c & 7) ^ (h & 7)) << 4);
     cp_async16(dst, h < H ? qrow + (size_t)h * D + c * 8 : qrow, h < H ? 16u : 0u);
   }
+  cp_async_commit();  // Q in a group of its own: the QK-norm prologue waits for Q alone
+  if ((a.qk_flags & kNrNorm) && tid < D)
+    sgam[tid] = a.q_gamma ? __bfloat162float(static_cast<const __nv_bfloat16 *>(a.q_gamma)[tid]) : 1.f;
   int t;
   bool ok = query_position(a.lens, a.q_pos, b, a.Tq, tq, t);
   int v = 0, w0 = 0, nwin = 0;
@@ -213,19 +217,13 @@ __global__ void __launch_bounds__(kAtThreads, 1) k_attend_tc(AttendArgs a) {
     } else if (pn < hi) {
       stage_ptrs(pn, kb ^ 1);  // while this tile's rows are in flight
     }
-    cp_async_wait_group<0>();
-    fence_proxy_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    if constexpr (NKB == 2) {
-      if (pn < hi) gather(pn, kb ^ 1);  // the next tile's rows during this tile's math
-    }
     if (a.qk_flags && p0 == lo) {
-      // QK-norm and partial RoPE of the staged query rows, in place, before
-      // the first S = Q K^T: this thread's 64 columns of head hrow are the 8
-      // swizzled 16-byte chunks of row hrow in Q atom `half`; the row's sum
-      // of squares is completed through the partner thread
+      // QK-norm and partial RoPE of the staged query rows, in place, while
+      // the first key tile is still in flight: this thread's 64 columns of
+      // head hrow are the 8 swizzled 16-byte chunks of row hrow in Q atom
+      // `half`; the row's sum of squares is completed through the partner
+      cp_async_wait_group<1>();  // Q's group (the older one) has landed
+      __syncthreads();
       const uint32_t qa = smem_u32(sQ) + half * kAtQAtom + hrow * 128;
       float ss = 0.f;
       if (hrow < H) {
@@ -246,9 +244,9 @@ __global__ void __launch_bounds__(kAtThreads, 1) k_attend_tc(AttendArgs a) {
       xmax[half][hrow] = ss;
       __syncthreads();
       ss += xmax[half ^ 1][hrow];
-      const float inv = (a.qk_flags & kNrNorm) ? 1.f / sqrtf(ss / (float)D + a.q_eps) : 1.f;
+      const bool nrm = (a.qk_flags & kNrNorm) != 0;
+      const float inv = nrm ? 1.f / sqrtf(ss / (float)D + a.q_eps) : 1.f;
       const int d0 = D - a.rope_r;
-      const __nv_bfloat16 *gq = (a.qk_flags & kNrNorm) ? static_cast<const __nv_bfloat16 *>(a.q_gamma) : nullptr;
       if (hrow < H) {
 #pragma unroll
         for (int cc = 0; cc < 8; ++cc) {
@@ -262,9 +260,9 @@ __global__ void __launch_bounds__(kAtThreads, 1) k_attend_tc(AttendArgs a) {
           for (int e = 0; e < 4; ++e) {
             const int col = half * (D / 2) + cc * 8 + 2 * e;
             float x0 = __uint_as_float(w[e] << 16) * inv, x1 = __uint_as_float(w[e] & 0xFFFF0000u) * inv;
-            if (gq) {
-              x0 *= __bfloat162float(gq[col]);
-              x1 *= __bfloat162float(gq[col + 1]);
+            if (nrm) {
+              x0 *= sgam[col];
+              x1 *= sgam[col + 1];
             }
             if ((a.qk_flags & kNrRotate) && col >= d0) rope_turn(x0, x1, rot_cs[(col - d0) >> 1], false);
             __nv_bfloat162 pr = __floats2bfloat162_rn(x0, x1);
@@ -275,8 +273,15 @@ __global__ void __launch_bounds__(kAtThreads, 1) k_attend_tc(AttendArgs a) {
                        : "memory");
         }
       }
-      fence_proxy_async_smem();
-      __syncthreads();
+      // made visible to the tensor core by the fence and barrier below
+    }
+    cp_async_wait_group<0>();
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if constexpr (NKB == 2) {
+      if (pn < hi) gather(pn, kb ^ 1);  // the next tile's rows during this tile's math
     }
     const uint32_t sKb = smem_u32(sK) + kb * 2 * kAtKHalf;
     // ---- S = Q K^T

@@ -960,7 +960,7 @@ int csa_norm_rope(const void *x, void *y, long R, int G, int d, const int32_t *p
   if (!x || !y) return fail(CSA_ERR_NULL, "%s: x and y must not be NULL", what);
   if (!aligned16(x) || !aligned16(y)) return fail(CSA_ERR_ALIGN, "%s: x and y must be 16-byte aligned", what);
   const long rows = R * (long)G;
-  if (rows / G != R || rows > (1L << 40)) return fail(CSA_ERR_UNSUPPORTED, "%s: too many rows", what);
+  if (rows / G != R || rows >= (1L << 31)) return fail(CSA_ERR_UNSUPPORTED, "%s: R*G >= 2^31 rows", what);
   csa::NormRopeArgs a;
   a.x = x;
   a.y = y;

@@ -357,8 +357,8 @@ CSA_API int hca_attend(const void *q, const void *kv_c, const void *kv_tok, int 
  *            stride m: pos_stride = m; a token array [B][Tq = n][d]:
  *            pos_stride = 1)
  *   eps    >= 0; rope_dim even, 0 <= rope_dim <= d; rope_base > 0
- * Supported: d in {64, 128}.  Caller owns every buffer; nothing is
- * allocated; asynchronous on `stream`.
+ * Supported: d in {64, 128}; R * G < 2^31.  Caller owns every buffer;
+ * nothing is allocated; asynchronous on `stream`.
  * ---------------------------------------------------------------------- */
 CSA_API int csa_norm_rope(const void *x, void *y, long R, int G, int d, const int32_t *pos,
                           const int32_t *lens, int Tq, int pos_stride, int pos_offset, const void *gamma,
