@@ -57,6 +57,8 @@ def _load():
         lib.orc_quantize_mxfp4.argtypes = [P, I, L, I, P, P]
         lib.orc_dequant_mxfp4.argtypes = [P, P, L, I, P]
         lib.orc_norm_rope.argtypes = [P, L, I, I, P, P, D, I, D, I, I, P]
+        lib.orc_quantize_fp8_entries.argtypes = [P, I, L, I, I, P, P, P]
+        lib.orc_dequant_fp8_entries.argtypes = [P, P, P, I, L, I, I, P]
         lib.orc_set_threads.argtypes = [I]
         lib.orc_get_threads.restype = I
         for name in ("orc_round", "orc_csa_compress", "orc_hca_compress", "orc_index_scores",
@@ -289,4 +291,37 @@ def norm_rope(x, pos, gamma=None, eps=1e-6, rope_dim=64, base=10000.0, norm=True
     flags = (1 if norm else 0) | (2 if rotate else 0) | (4 if inverse else 0)
     _check(_load().orc_norm_rope(px, R, G, d, p.ctypes.data, pg, float(eps), int(rope_dim),
                                  float(base), flags, dt, out.ctypes.data), "norm_rope")
+    return out
+
+
+def quantize_fp8_entries(x, rope_dim=64):
+    """Entries ``x`` ``[..., d]`` -> (fp8 codes ``[..., d - r]`` uint8, UE8M0
+    scales ``[..., (d - r) / 64]`` uint8, rope dims ``[..., r]`` in x's
+    dtype): the FP8 cache entry read stated at ``orc_quantize_fp8_entries``."""
+    dt = _dt_of(x)
+    *lead, d = x.shape
+    rows = int(np.prod(lead)) if lead else 1
+    q = d - rope_dim
+    xc, px = _c(x)
+    fp8 = np.zeros((*lead, q), np.uint8)
+    sc = np.zeros((*lead, q // 64), np.uint8)
+    rope = np.zeros((*lead, rope_dim), x.dtype)
+    _check(_load().orc_quantize_fp8_entries(px, dt, rows, d, int(rope_dim), fp8.ctypes.data, sc.ctypes.data,
+                                            rope.ctypes.data), "quantize_fp8_entries")
+    return fp8, sc, rope
+
+
+def dequant_fp8_entries(fp8, scales, rope):
+    """Exact float64 values of FP8 entries (inverse layout of
+    ``quantize_fp8_entries``)."""
+    dt = _dt_of(rope)
+    *lead, q = fp8.shape
+    r = rope.shape[-1]
+    d = q + r
+    rows = int(np.prod(lead)) if lead else 1
+    f, pf = _c(fp8, np.uint8)
+    s_, ps = _c(scales, np.uint8)
+    rp, pr = _c(rope)
+    out = np.empty((*lead, d), np.float64)
+    _check(_load().orc_dequant_fp8_entries(pf, ps, pr, dt, rows, d, r, out.ctypes.data), "dequant_fp8_entries")
     return out

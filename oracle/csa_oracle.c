@@ -630,3 +630,102 @@ int orc_norm_rope(const void *x, long R, int G, int d, const int64_t *pos, const
   }
   return ORC_OK;
 }
+
+/* ------------------------------------------------------------------ */
+/* FP8 cache entries                                                   */
+/* ------------------------------------------------------------------ */
+
+/*
+ * [A4] "The KV cache, recomputed": an entry keeps its 64 RoPE dimensions in
+ * BF16 and the other dimensions in FP8, with one-byte UE8M0 scales (448 FP8
+ * numbers and 7 scales: one scale per 64 numbers).  Reading: the FP8 format
+ * is E4M3 (sign, 4 exponent bits of bias 7, 3 mantissa bits; subnormals
+ * m/8 * 2^-6; largest finite 1.75 * 2^8 = 448; the code S.1111.111 is NaN),
+ * the scale rule the one of the MXFP4 keys above: per block of 64 elements
+ * X = floor(log2 amax) - 8 (8: the exponent of 448), clamped to
+ * [-127, 127], X = -127 for an all-zero block, stored as X + 127; each
+ * element becomes the E4M3 value nearest to x / 2^X, ties to the code with
+ * an even mantissa, magnitudes above 448 saturate to 448, the sign of -0.0
+ * is kept.  The last `r` dims (the rotated ones) are copied unchanged.
+ * Layout: fp8 [rows][d - r] codes, scales [rows][(d - r) / 64], rope
+ * [rows][r] in the input dtype.  Dequantised value: code value * 2^X.
+ */
+static double e4m3_value(int code) { /* code 0..126, the sign bit clear */
+  const int e = (code >> 3) & 15, m = code & 7;
+  return e == 0 ? ldexp((double)m, -9) : ldexp(1.0 + m / 8.0, e - 7);
+}
+
+/* nearest E4M3 magnitude code of y >= 0 (brute force over the 127 finite
+ * codes, ascending in value), ties to the even code, saturating at 448 */
+static int e4m3_code(double y) {
+  if (y >= 448.0) return 126;
+  int best = 0;
+  double bd = INFINITY;
+  for (int c = 0; c <= 126; ++c) {
+    const double dd = fabs(e4m3_value(c) - y);
+    if (dd < bd || (dd == bd && (c % 2) == 0)) {
+      bd = dd;
+      best = c;
+    }
+  }
+  return best;
+}
+
+int orc_quantize_fp8_entries(const void *x, int dt, long rows, int d, int r, uint8_t *fp8, uint8_t *scales,
+                             void *rope) {
+  const int q = d - r;
+  if (!x || rows < 0 || d <= 0 || r < 0 || r > d || q % 64) return ORC_ERR_ARG;
+  if ((q > 0 && (!fp8 || !scales)) || (r > 0 && !rope)) return ORC_ERR_ARG;
+  if (dt != ORC_F32 && dt != ORC_BF16) return ORC_ERR_ARG;
+#pragma omp parallel for schedule(static)
+  for (long row = 0; row < rows; ++row) {
+    for (int blk = 0; blk < q / 64; ++blk) {
+      double amax = 0.0;
+      for (int e = 0; e < 64; ++e) {
+        const double v = fabs(ld(x, dt, (size_t)row * d + blk * 64 + e));
+        if (v > amax) amax = v;
+      }
+      int X = -127;
+      if (amax > 0.0) {
+        int ex;
+        (void)frexp(amax, &ex); /* floor(log2 amax) = ex - 1 */
+        X = ex - 1 - 8;
+        if (X < -127) X = -127;
+        if (X > 127) X = 127;
+      }
+      scales[(size_t)row * (q / 64) + blk] = (uint8_t)(X + 127);
+      for (int e = 0; e < 64; ++e) {
+        const double v = ld(x, dt, (size_t)row * d + blk * 64 + e);
+        int c = e4m3_code(ldexp(fabs(v), -X));
+        if (signbit(v)) c |= 0x80;
+        fp8[(size_t)row * q + blk * 64 + e] = (uint8_t)c;
+      }
+    }
+    for (int e = 0; e < r; ++e) {
+      if (dt == ORC_F32)
+        ((float *)rope)[(size_t)row * r + e] = ((const float *)x)[(size_t)row * d + q + e];
+      else
+        ((uint16_t *)rope)[(size_t)row * r + e] = ((const uint16_t *)x)[(size_t)row * d + q + e];
+    }
+  }
+  return ORC_OK;
+}
+
+/* fp8 / scales / rope as above -> out [rows][d] double (exact values) */
+int orc_dequant_fp8_entries(const uint8_t *fp8, const uint8_t *scales, const void *rope, int dt, long rows,
+                            int d, int r, double *out) {
+  const int q = d - r;
+  if (!out || rows < 0 || d <= 0 || r < 0 || r > d || q % 64) return ORC_ERR_ARG;
+  if ((q > 0 && (!fp8 || !scales)) || (r > 0 && !rope)) return ORC_ERR_ARG;
+  for (long row = 0; row < rows; ++row) {
+    for (int e = 0; e < q; ++e) {
+      const int c = fp8[(size_t)row * q + e];
+      const int X = (int)scales[(size_t)row * (q / 64) + e / 64] - 127;
+      if ((c & 0x7F) == 0x7F) return ORC_ERR_ARG; /* NaN codes are never produced */
+      const double v = ldexp(e4m3_value(c & 0x7F), X);
+      out[(size_t)row * d + e] = (c & 0x80) ? -v : v;
+    }
+    for (int e = 0; e < r; ++e) out[(size_t)row * d + q + e] = ld(rope, dt, (size_t)row * r + e);
+  }
+  return ORC_OK;
+}

@@ -17,7 +17,7 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 SRC = os.path.join(ROOT, "oracle", "csa_oracle.c")
 PINS = ["tests/test_oracle_compress.py", "tests/test_oracle_index_topk.py",
         "tests/test_oracle_attend.py", "tests/test_oracle_e2e.py",
-        "tests/test_oracle_mxfp4.py", "tests/test_oracle_rope.py"]
+        "tests/test_oracle_mxfp4.py", "tests/test_oracle_rope.py", "tests/test_oracle_fp8.py"]
 
 MUTANTS = {
     "csa_series_swapped": ("const void *W = (j < 4) ? Wa : Wb;", "const void *W = (j < 4) ? Wb : Wa;"),
@@ -50,6 +50,10 @@ MUTANTS = {
     "rope_half_split_pairs": ("const int i0 = d - r + 2 * j, i1 = i0 + 1;", "const int i0 = d - r + j, i1 = i0 + r / 2;"),
     "rope_frequency_exponent": ("pow(base, -2.0 * j / r)", "pow(base, -1.0 * j / r)"),
     "rope_inverse_ignored": ("(flags & 4) ? -(double)pos[rr] : (double)pos[rr]", "(double)pos[rr]"),
+    "fp8_ties_to_odd": ("if (dd < bd || (dd == bd && (c % 2) == 0)) {", "if (dd < bd || (dd == bd && (c % 2) == 1)) {"),
+    "fp8_scale_off_by_one": ("X = ex - 1 - 8;", "X = ex - 1 - 7;"),
+    "fp8_rope_dims_misplaced": ("((uint16_t *)rope)[(size_t)row * r + e] = ((const uint16_t *)x)[(size_t)row * d + q + e];",
+                                "((uint16_t *)rope)[(size_t)row * r + e] = ((const uint16_t *)x)[(size_t)row * d + e];"),
     "round_double_rounding": ("r = nearbyint(ldexp(a, -q));", "r = nearbyint(ldexp((double)(float)a, -q));"),
 }
 
