@@ -72,6 +72,9 @@ def lib() -> ctypes.CDLL:
         L.csa_attend.argtypes = [P, P, P, I, P, P, P, I, I, I, I, I, I, I, F, P, I, P, P]
         L.hca_attend.argtypes = [P, P, P, I, P, P, I, I, I, I, I, I, I, F, P, I, P, P]
         L.csa_norm_rope.argtypes = [P, P, ctypes.c_long, I, I, P, P, I, I, I, P, F, I, F, I, I, P]
+        L.csa_quantize_fp8_entries.argtypes = [P, ctypes.c_long, I, I, I, P, P, P, P]
+        L.csa_attend_fp8.argtypes = [P, P, P, P, P, I, P, P, P, I, I, I, I, I, I, I, F, P, I, P, P]
+        L.hca_attend_fp8.argtypes = [P, P, P, P, P, I, P, P, I, I, I, I, I, I, I, F, P, I, P, P]
         L.csa_attend_rope.argtypes = [P, P, P, I, P, P, P, I, I, I, I, I, I, I, F, P, P, F, I, F, I, I, P, P]
         L.hca_attend_rope.argtypes = [P, P, P, I, P, P, I, I, I, I, I, I, I, F, P, P, F, I, F, I, I, P, P]
         for name in ("csa_check_device_error", "csa_compress", "hca_compress", "csa_compress_step",
@@ -377,4 +380,45 @@ def hca_attend_rope(q, kv_c, kv_tok, lens, q_pos=None, m=128, window=128, scale=
                                  B, Tq, H, d, kv_c.shape[1], m, window, float(scale), _f32(sink),
                                  _p(q_gamma), float(eps), int(rope_dim), float(rope_base), int(flags), _dt(q),
                                  _p(out), _s(stream)))
+    return out
+
+
+def csa_quantize_fp8_entries(kv, rope_dim=64, stream=None):
+    """Entries kv [..., d] -> (E4M3 codes [..., d - rope_dim] uint8, UE8M0
+    scales [..., (d - rope_dim) / 64] uint8, the last rope_dim dims [..., rope_dim])."""
+    *lead, d = kv.shape
+    rows = 1
+    for n in lead:
+        rows *= n
+    q = d - rope_dim
+    fp8 = torch.empty(*lead, q, dtype=torch.uint8, device=kv.device)
+    sc = torch.empty(*lead, q // 64, dtype=torch.uint8, device=kv.device)
+    rope = torch.empty(*lead, rope_dim, dtype=kv.dtype, device=kv.device)
+    _check(lib().csa_quantize_fp8_entries(_p(kv), rows, d, int(rope_dim), _dt(kv), _u8(fp8), _u8(sc), _p(rope),
+                                          _s(stream)))
+    return fp8, sc, rope
+
+
+def csa_attend_fp8(q, kv_fp8, kv_scales, kv_rope, kv_tok, idx, lens, q_pos=None, window=128, scale=0.0, out=None,
+                   stream=None, sink=None):
+    """csa_attend over FP8 entries: kv_fp8 [B][nc_max][64] uint8, kv_scales
+    [B][nc_max] (or [B][nc_max][1]) uint8, kv_rope [B][nc_max][64] bf16."""
+    B, Tq, H, d = q.shape
+    if out is None:
+        out = torch.empty_like(q)
+    _check(lib().csa_attend_fp8(_p(q), _u8(kv_fp8), _u8(kv_scales), _p(kv_rope), _p(kv_tok), kv_tok.shape[1],
+                                _i32(idx), _i32(lens), _i32(q_pos), B, Tq, H, d, kv_fp8.shape[1], idx.shape[-1],
+                                window, float(scale), _f32(sink), _dt(q), _p(out), _s(stream)))
+    return out
+
+
+def hca_attend_fp8(q, kv_fp8, kv_scales, kv_rope, kv_tok, lens, q_pos=None, m=128, window=128, scale=0.0,
+                   out=None, stream=None, sink=None):
+    """hca_attend over FP8 entries (planes as csa_attend_fp8)."""
+    B, Tq, H, d = q.shape
+    if out is None:
+        out = torch.empty_like(q)
+    _check(lib().hca_attend_fp8(_p(q), _u8(kv_fp8), _u8(kv_scales), _p(kv_rope), _p(kv_tok), kv_tok.shape[1],
+                                _i32(lens), _i32(q_pos), B, Tq, H, d, kv_fp8.shape[1], m, window, float(scale),
+                                _f32(sink), _dt(q), _p(out), _s(stream)))
     return out

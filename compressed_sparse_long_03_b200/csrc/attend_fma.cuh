@@ -56,6 +56,12 @@ struct AttendArgs {
   const void *q_gamma;
   float q_eps;
   double rope_log2_base;
+  // FP8 cache entries (tensor-core kernel, d = 128): the first 64 dims as
+  // E4M3 codes [B][nc_max][64] with one UE8M0 scale byte per entry
+  // [B][nc_max], the last 64 dims in bf16 [B][nc_max][64]; nullptr: kv_c
+  const uint8_t *kv_fp8;
+  const uint8_t *kv_sc;
+  const void *kv_rope;
 };
 
 // Round a float to the storage type T (what a staged query holds).

@@ -31,6 +31,7 @@
 
 #include "attend_fma.cuh"
 #include "common.cuh"
+#include "fp8.cuh"
 #include "sm100.cuh"
 
 namespace csa {
@@ -41,11 +42,17 @@ constexpr uint32_t kAtQAtom = 128 * 128;             // 128 rows x 128 B
 constexpr uint32_t kAtKHalf = kAtMaxTile * 128;      // one 64-wide d slice of the key tile
 constexpr uint32_t kAtPAtom = 128 * 128;             // 128 heads x 64 keys x 2 B
 constexpr uint32_t kAtPart = 128 * 128 * 4;          // partial outputs pushed by the cluster
+constexpr uint32_t kAtF8Rows = kAtMaxTile * 64 + kAtMaxTile * 4;  // raw codes + scale words of a tile
 // Dynamic shared memory: Q, the key tile (two, double-buffered, for one-CTA
-// rows), P, and for clusters the partials pushed by the peers.
-__host__ __device__ constexpr size_t at_smem_bytes(int cs) {
+// rows), P, for clusters the partials pushed by the peers, and with FP8
+// entries the tiles' raw codes and scale words.
+__host__ __device__ constexpr size_t at_smem_bytes(int cs, bool fp8 = false) {
   return 1024 + 2 * kAtQAtom + (cs == 1 ? 2 : 1) * 2 * kAtKHalf + (kAtMaxTile / 64) * kAtPAtom +
-         (cs == 1 ? 0 : kAtPart);
+         (cs == 1 ? 0 : kAtPart) + (fp8 ? (cs == 1 ? 2 : 1) * kAtF8Rows : 0);
+}
+
+__device__ __forceinline__ void at_cp_async4(uint32_t dst, const void *src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
 }
 
 template <int CS>
@@ -58,6 +65,7 @@ __global__ void __launch_bounds__(kAtThreads, 1) k_attend_tc(AttendArgs a) {
   constexpr int NKB = CS == 1 ? 2 : 1;  // key-tile buffers
   __shared__ int kvalid[NKB][kAtMaxTile / 32];  // validity bits, one word per 32 keys
   __shared__ const __nv_bfloat16 *rowp[NKB][kAtMaxTile];
+  __shared__ int rowe[NKB][kAtMaxTile];  // FP8 entries: the entry's row in the cache planes, else -1
   __shared__ float pm[136], pl[136];   // pushed partial max / sum [hl * CS + c]
   __shared__ float xmax[2][128];       // per-half row max (then sum) of the partner
   __shared__ float mw[136], minv[128];  // merge weights [hl * CS + c], 1 / sum
@@ -73,6 +81,11 @@ __global__ void __launch_bounds__(kAtThreads, 1) k_attend_tc(AttendArgs a) {
   // partials of the heads this CTA finalises, written by every CTA of the
   // cluster: [head slot hl][source rank c][128] (slot hl = head h / CS)
   float *part = reinterpret_cast<float *>(sP + (kAtMaxTile / 64) * kAtPAtom);
+  // FP8 entries: raw codes [NKB][tile rows][64 B], then scale words [NKB][tile rows]
+  uint8_t *sF8 = reinterpret_cast<uint8_t *>(part) + (CS == 1 ? 0 : kAtPart);
+  uint32_t *sF8s = reinterpret_cast<uint32_t *>(sF8 + NKB * kAtMaxTile * 64);
+  const bool f8 = a.kv_fp8 != nullptr;
+  const __nv_bfloat16 *kv_rp = static_cast<const __nv_bfloat16 *>(a.kv_rope);
 
   const int rank = (CS > 1) ? (int)cg::this_cluster().block_rank() : 0;
   const int r = blockIdx.x / CS;
@@ -169,16 +182,25 @@ __global__ void __launch_bounds__(kAtThreads, 1) k_attend_tc(AttendArgs a) {
     for (int j = tid; j < nc * 32; j += kAtThreads) {
       const int p = p0 + j;
       const __nv_bfloat16 *row = nullptr;
+      int e = -1;
       if (j < nt) {
         if (p < nsel) {
           const int i = a.idx ? __ldg(a.idx + (size_t)r * a.k + p) : p;
-          if (i >= 0 && i < v) row = kv_c + ((size_t)b * a.nc_max + i) * D;
+          if (i >= 0 && i < v) {
+            if (f8) {
+              e = b * a.nc_max + i;
+              row = kv_rp + (size_t)e * (D / 2);
+            } else {
+              row = kv_c + ((size_t)b * a.nc_max + i) * D;
+            }
+          }
         } else {
           const int s = w0 + (p - nsel);
           row = kv_tok + ((size_t)b * a.n_tok + (s % a.n_tok)) * D;
         }
       }
       rowp[kb][j] = row;
+      rowe[kb][j] = e;
       // a warp covers 32 consecutive keys: one validity word per 32
       const unsigned vm = __ballot_sync(0xffffffffu, row != nullptr);
       if ((tid & 31) == 0) kvalid[kb][j >> 5] = (int)vm;
@@ -192,8 +214,17 @@ __global__ void __launch_bounds__(kAtThreads, 1) k_attend_tc(AttendArgs a) {
     for (int u = tid; u < nc * 32 * 16; u += kAtThreads) {
       const int j = u >> 4, c = u & 15;
       const __nv_bfloat16 *row = rowp[kb][j];
-      cp_async16(k0 + (c >> 3) * kAtKHalf + j * 128 + (((c & 7) ^ (j & 7)) << 4), row ? row + c * 8 : kv_tok,
-                 row ? 16u : 0u);
+      const uint32_t dst = k0 + (c >> 3) * kAtKHalf + j * 128 + (((c & 7) ^ (j & 7)) << 4);
+      const int e = f8 ? rowe[kb][j] : -1;
+      if (e < 0) {
+        cp_async16(dst, row ? row + c * 8 : kv_tok, row ? 16u : 0u);
+      } else if (c >= 8) {  // the bf16 (rotated) half of an FP8 entry, straight into the tile
+        cp_async16(dst, row + (c - 8) * 8, 16u);
+      } else if (c < 4) {   // its 64 codes, raw, widened once the tile has landed
+        cp_async16(smem_u32(sF8) + (kb * kAtMaxTile + j) * 64 + c * 16, a.kv_fp8 + (size_t)e * 64 + c * 16, 16u);
+      } else if (c == 4) {  // the aligned word holding its scale byte
+        at_cp_async4(smem_u32(sF8s + kb * kAtMaxTile + j), a.kv_sc + (e & ~3));
+      }
     }
     cp_async_commit();
   };
@@ -284,6 +315,25 @@ __global__ void __launch_bounds__(kAtThreads, 1) k_attend_tc(AttendArgs a) {
       if (pn < hi) gather(pn, kb ^ 1);  // the next tile's rows during this tile's math
     }
     const uint32_t sKb = smem_u32(sK) + kb * 2 * kAtKHalf;
+    if (f8) {
+      // widen the FP8 entries' codes into the tile's first 64 dims: 8 codes
+      // (16 B of bf16, one swizzled chunk) per thread and step
+      for (int u = tid; u < nchunk * 32 * 8; u += kAtThreads) {
+        const int j = u >> 3, c = u & 7;
+        const int e = rowe[kb][j];
+        if (e < 0) continue;
+        const uint32_t sw = sF8s[kb * kAtMaxTile + j];
+        const int X = (int)((sw >> (8 * (e & 3))) & 0xFFu) - 127;
+        const uint2 raw = *reinterpret_cast<const uint2 *>(sF8 + (kb * kAtMaxTile + j) * 64 + c * 8);
+        uint32_t w[4];
+        f8_widen8(raw.x, raw.y, f8_pow2(X), w);
+        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(sKb + j * 128 + ((c ^ (j & 7)) << 4)),
+                     "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3])
+                     : "memory");
+      }
+      fence_proxy_async_smem();
+      __syncthreads();
+    }
     // ---- S = Q K^T
     if (tid == 0) {
       const uint32_t idesc = idesc_bf16_f32(128, 32 * nchunk);

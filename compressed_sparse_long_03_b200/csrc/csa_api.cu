@@ -30,6 +30,7 @@
 #include "topk.cuh"
 #include "attend_fma.cuh"
 #include "attend_tc.cuh"
+#include "fp8.cuh"
 #include "rope.cuh"
 
 namespace {
@@ -576,7 +577,7 @@ int launch_attend_tc(const csa::AttendArgs &a, int R, cudaStream_t st, const cha
     case 4: kern = csa::k_attend_tc<4>; break;
     default: kern = csa::k_attend_tc<8>; break;
   }
-  const size_t smem = csa::at_smem_bytes(cs);
+  const size_t smem = csa::at_smem_bytes(cs, a.kv_fp8 != nullptr);
   int rc = ensure_smem(kern, smem, what);
   if (rc) return rc;
   return launch_cluster(kern, cs, (unsigned)cs * R, csa::kAtThreads, smem, st, what, a);
@@ -589,6 +590,13 @@ struct QkSpec {
   float eps = 0.f;
   int rope_dim = 0;
   float rope_base = 0.f;
+};
+
+// FP8 entry planes of csa_attend_fp8 / hca_attend_fp8 (all NULL: kv_c).
+struct F8Spec {
+  const uint8_t *codes = nullptr;
+  const uint8_t *scales = nullptr;
+  const void *rope = nullptr;
 };
 
 // Validation shared by csa_norm_rope and the fused attention.
@@ -613,9 +621,20 @@ int attend_common(const void *q, const void *kv_c, const void *kv_tok, int n_tok
                   const int32_t *idx, const int32_t *lens, const int32_t *q_pos, int B, int Tq,
                   int H, int d, int nc_max, int k, int m, int window, float scale,
                   const float *sink, csa_dtype dt, void *out, void *stream, const char *what,
-                  const QkSpec &qk = QkSpec()) {
+                  const QkSpec &qk = QkSpec(), const F8Spec &f8 = F8Spec()) {
   int rc = check_dtype(dt, what);
   if (rc) return rc;
+  const bool fp8 = f8.codes || f8.scales || f8.rope;
+  if (fp8) {
+    if (dt != CSA_BF16 || d != 128)
+      return fail(CSA_ERR_UNSUPPORTED, "%s: FP8 entries need bf16 and d = 128 (64 FP8 + 64 bf16 dims)", what);
+    if (nc_max % 4) return fail(CSA_ERR_UNSUPPORTED, "%s: FP8 entries need nc_max %% 4 == 0", what);
+    if (nc_max > 0 && (!f8.codes || !f8.scales || !f8.rope))
+      return fail(CSA_ERR_NULL, "%s: an FP8 entry plane is NULL", what);
+    if (nc_max > 0 && (!aligned16(f8.codes) || !aligned16(f8.rope) || (reinterpret_cast<uintptr_t>(f8.scales) & 3)))
+      return fail(CSA_ERR_ALIGN, "%s: FP8 codes and rope planes 16-byte aligned, scales 4-byte", what);
+    if ((long)B * nc_max >= (1L << 31)) return fail(CSA_ERR_UNSUPPORTED, "%s: B * nc_max >= 2^31", what);
+  }
   if (qk.flags) {
     if (qk.flags & CSA_NR_INVERSE)
       return fail(CSA_ERR_UNSUPPORTED, "%s: the output's inverse rotation follows CSA_NR_ROTATE", what);
@@ -624,7 +643,7 @@ int attend_common(const void *q, const void *kv_c, const void *kv_tok, int n_tok
   }
   if (B < 0 || Tq < 0) return fail(CSA_ERR_SHAPE, "%s: B=%d and Tq=%d must be >= 0", what, B, Tq);
   if ((long)B * Tq == 0) return CSA_OK;
-  if (!q || !kv_tok || !lens || !out || (idx == nullptr && k > 0) || (nc_max > 0 && !kv_c))
+  if (!q || !kv_tok || !lens || !out || (idx == nullptr && k > 0) || (nc_max > 0 && !kv_c && !fp8))
     return fail(CSA_ERR_NULL, "%s: a required pointer is NULL", what);
   if (!aligned16(q) || !aligned16(kv_tok) || !aligned16(out) || (kv_c && !aligned16(kv_c)))
     return fail(CSA_ERR_ALIGN, "%s: tensors must be 16-byte aligned", what);
@@ -658,6 +677,9 @@ int attend_common(const void *q, const void *kv_c, const void *kv_tok, int n_tok
   a.q_gamma = (qk.flags & CSA_NR_NORM) ? qk.gamma : nullptr;
   a.q_eps = qk.eps;
   a.rope_log2_base = (qk.flags & CSA_NR_ROTATE) ? std::log2((double)qk.rope_base) : 0.0;
+  a.kv_fp8 = fp8 ? f8.codes : nullptr;
+  a.kv_sc = fp8 ? f8.scales : nullptr;
+  a.kv_rope = fp8 ? f8.rope : nullptr;
   const int R = B * Tq;
   const long max_keys = (idx ? (long)k : (long)nc_max) + window;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -940,6 +962,61 @@ int hca_attend(const void *q, const void *kv_c, const void *kv_tok, int n_tok,
   if (nc_max > 65536) return fail(CSA_ERR_UNSUPPORTED, "hca_attend: nc_max=%d > 65536", nc_max);
   return attend_common(q, kv_c, kv_tok, n_tok, nullptr, lens, q_pos, B, Tq, H, d, nc_max, 0, m,
                        window, scale, sink, dt, out, stream, "hca_attend");
+}
+
+int csa_quantize_fp8_entries(const void *kv, long rows, int d, int rope_dim, csa_dtype dt, uint8_t *fp8,
+                             uint8_t *scales, void *rope, void *stream) {
+  const char *what = "csa_quantize_fp8_entries";
+  begin_call();
+  int rc = check_dtype(dt, what);
+  if (rc) return rc;
+  if (d < 64 || d > 4096 || rope_dim < 0 || rope_dim > d || (d - rope_dim) % 64 || (rope_dim & 1))
+    return fail(CSA_ERR_UNSUPPORTED, "%s: d=%d, rope_dim=%d: d - rope_dim must be a multiple of 64", what, d,
+                rope_dim);
+  if (rows < 0 || rows >= (1L << 31)) return fail(CSA_ERR_SHAPE, "%s: rows=%ld not in [0, 2^31)", what, rows);
+  if (rows == 0) return CSA_OK;
+  if (!kv || (d > rope_dim && (!fp8 || !scales)) || (rope_dim > 0 && !rope))
+    return fail(CSA_ERR_NULL, "%s: a required pointer is NULL", what);
+  if (!aligned16(kv) || (fp8 && (reinterpret_cast<uintptr_t>(fp8) & 1)) || (rope && !aligned16(rope)))
+    return fail(CSA_ERR_ALIGN, "%s: kv and rope 16-byte aligned, fp8 2-byte aligned", what);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const unsigned grid = (unsigned)std::max(1L, std::min((rows + 7) / 8, 8L * num_sms()));
+  if (dt == CSA_F32)
+    return launch_cluster(csa::k_quantize_fp8_entries<float>, 1, grid, csa::kF8Threads, 0, st, what,
+                          static_cast<const float *>(kv), rows, d, rope_dim, fp8, scales, static_cast<float *>(rope));
+  return launch_cluster(csa::k_quantize_fp8_entries<__nv_bfloat16>, 1, grid, csa::kF8Threads, 0, st, what,
+                        static_cast<const __nv_bfloat16 *>(kv), rows, d, rope_dim, fp8, scales,
+                        static_cast<__nv_bfloat16 *>(rope));
+}
+
+int csa_attend_fp8(const void *q, const uint8_t *kv_fp8, const uint8_t *kv_scales, const void *kv_rope,
+                   const void *kv_tok, int n_tok, const int32_t *idx, const int32_t *lens, const int32_t *q_pos,
+                   int B, int Tq, int H, int d, int nc_max, int k, int window, float scale, const float *sink,
+                   csa_dtype dt, void *out, void *stream) {
+  begin_call();
+  if (k < 1 || k > 4096) return fail(CSA_ERR_UNSUPPORTED, "csa_attend_fp8: k=%d not in [1,4096]", k);
+  if (!idx && (long)B * Tq > 0) return fail(CSA_ERR_NULL, "csa_attend_fp8: idx is NULL");
+  F8Spec f8;
+  f8.codes = kv_fp8;
+  f8.scales = kv_scales;
+  f8.rope = kv_rope;
+  return attend_common(q, nullptr, kv_tok, n_tok, idx, lens, q_pos, B, Tq, H, d, nc_max, k, 4, window, scale,
+                       sink, dt, out, stream, "csa_attend_fp8", QkSpec(), f8);
+}
+
+int hca_attend_fp8(const void *q, const uint8_t *kv_fp8, const uint8_t *kv_scales, const void *kv_rope,
+                   const void *kv_tok, int n_tok, const int32_t *lens, const int32_t *q_pos, int B, int Tq, int H,
+                   int d, int nc_max, int m, int window, float scale, const float *sink, csa_dtype dt, void *out,
+                   void *stream) {
+  begin_call();
+  if (m < 1 || m > 4096) return fail(CSA_ERR_UNSUPPORTED, "hca_attend_fp8: m=%d not in [1,4096]", m);
+  if (nc_max > 65536) return fail(CSA_ERR_UNSUPPORTED, "hca_attend_fp8: nc_max=%d > 65536", nc_max);
+  F8Spec f8;
+  f8.codes = kv_fp8;
+  f8.scales = kv_scales;
+  f8.rope = kv_rope;
+  return attend_common(q, nullptr, kv_tok, n_tok, nullptr, lens, q_pos, B, Tq, H, d, nc_max, 0, m, window,
+                       scale, sink, dt, out, stream, "hca_attend_fp8", QkSpec(), f8);
 }
 
 int csa_norm_rope(const void *x, void *y, long R, int G, int d, const int32_t *pos, const int32_t *lens,

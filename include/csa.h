@@ -386,6 +386,46 @@ CSA_API int hca_attend_rope(const void *q, const void *kv_c, const void *kv_tok,
                             int m, int window, float scale, const float *sink, const void *q_gamma, float eps,
                             int rope_dim, float rope_base, int flags, csa_dtype dt, void *out, void *stream);
 
+/* ------------------------------------------------------------------------
+ * FP8 cache entries.
+ *
+ * Anatomy page, "The KV cache, recomputed": an entry keeps its 64 RoPE
+ * dimensions in BF16 and the others in FP8 with one-byte UE8M0 scales (448
+ * numbers and 7 scales: one per 64).  Reading: E4M3 codes (largest finite
+ * 448); per block of 64 elements the scale 2^X with X = floor(log2 amax) - 8
+ * clamped to [-127, 127] (-127 for an all-zero block), stored as the byte
+ * X + 127; each element x / 2^X rounded to the nearest E4M3 value, ties to
+ * even, saturating at 448.  The pages pack one record per entry; here the
+ * entry is held in three planes:
+ *   fp8    [rows][d - rope_dim]         E4M3 codes
+ *   scales [rows][(d - rope_dim) / 64]  UE8M0 bytes
+ *   rope   [rows][rope_dim]             the last rope_dim dims, unchanged
+ * A dequantised element (code value * 2^X) is exact in bf16.
+ * ---------------------------------------------------------------------- */
+
+/* csa_quantize_fp8_entries -- kv [rows][d] (dt) into the three planes.
+ * Supported: d - rope_dim a positive multiple of 64 (or 0), rope_dim even;
+ * rows < 2^31.  kv and rope 16-byte aligned, fp8 2-byte aligned. */
+CSA_API int csa_quantize_fp8_entries(const void *kv, long rows, int d, int rope_dim, csa_dtype dt, uint8_t *fp8,
+                                     uint8_t *scales, void *rope, void *stream);
+
+/* csa_attend_fp8 / hca_attend_fp8 -- csa_attend / hca_attend over a cache
+ * of FP8 entries (planes of csa_quantize_fp8_entries with rows = B * nc_max,
+ * d = 128, rope_dim = 64): the attention over the entries' dequantised
+ * values.  The tensor-core kernel widens the codes in shared memory as the
+ * tiles land.  Window tokens stay bf16.  Supported: bf16, d = 128,
+ * nc_max % 4 == 0 (the scales are fetched in aligned 4-byte words); other
+ * arguments as csa_attend / hca_attend.
+ * ---------------------------------------------------------------------- */
+CSA_API int csa_attend_fp8(const void *q, const uint8_t *kv_fp8, const uint8_t *kv_scales, const void *kv_rope,
+                           const void *kv_tok, int n_tok, const int32_t *idx, const int32_t *lens,
+                           const int32_t *q_pos, int B, int Tq, int H, int d, int nc_max, int k, int window,
+                           float scale, const float *sink, csa_dtype dt, void *out, void *stream);
+CSA_API int hca_attend_fp8(const void *q, const uint8_t *kv_fp8, const uint8_t *kv_scales, const void *kv_rope,
+                           const void *kv_tok, int n_tok, const int32_t *lens, const int32_t *q_pos, int B, int Tq,
+                           int H, int d, int nc_max, int m, int window, float scale, const float *sink,
+                           csa_dtype dt, void *out, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

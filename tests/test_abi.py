@@ -159,3 +159,26 @@ def test_norm_rope_validation(L):
     rc = L.hca_attend_rope(A16, A16, A16, 128, A16, None, 1, 1, 4, 128, 8, 128, 128, ctypes.c_float(0.0),
                            None, None, ctypes.c_float(1e-6), 63, ctypes.c_float(1e4), 2, 1, A16, None)
     assert rc == E_UNSUP
+
+
+def test_fp8_entries_validation(L):
+    q8 = L.csa_quantize_fp8_entries
+    assert q8(A16, 4, 100, 64, 1, A16, A16, A16, None) == E_UNSUP       # 36 FP8 dims
+    assert q8(A16, 4, 128, 63, 1, A16, A16, A16, None) == E_UNSUP
+    assert q8(A16, -1, 128, 64, 1, A16, A16, A16, None) == E_SHAPE
+    assert q8(None, 4, 128, 64, 1, A16, A16, A16, None) == E_NULL
+    assert q8(A4, 4, 128, 64, 1, A16, A16, A16, None) == E_ALIGN
+    assert q8(A16, 0, 128, 64, 1, A16, A16, A16, None) == OK
+
+    def att(fn="csa_attend_fp8", d=128, nc=8, dt=1, codes=A16, scales=A16, rope=A16):
+        if fn == "csa_attend_fp8":
+            return L.csa_attend_fp8(A16, codes, scales, rope, A16, 128, A16, A16, None, 1, 1, 4, d, nc, 4, 128,
+                                    ctypes.c_float(0.0), None, dt, A16, None)
+        return L.hca_attend_fp8(A16, codes, scales, rope, A16, 128, A16, None, 1, 1, 4, d, nc, 128, 128,
+                                ctypes.c_float(0.0), None, dt, A16, None)
+    assert att(d=64) == E_UNSUP
+    assert att(dt=0) == E_UNSUP
+    assert att(nc=6) == E_UNSUP
+    assert att(codes=None) == E_NULL
+    assert att(rope=A4) == E_ALIGN
+    assert att("hca_attend_fp8", nc=65540) == E_UNSUP
