@@ -46,11 +46,11 @@ def parse():
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-steps", type=int, default=1, help="oracle steps for cpu_baseline")
-    p.add_argument("--workload", type=int, default=4, choices=[1, 2, 3, 4, 5, 6, 7],
+    p.add_argument("--workload", type=int, default=4, choices=[1, 2, 3, 4, 5, 6, 7, 8],
                    help="4 (default): the 1M CSA decode step; 1, 2, 3, 5: the other "
                         "workloads, one measurement line each (single GPU); 6: workload 4 "
                         "with its indexer keys in MXFP4; 7: workload 4 with QK-norm and "
-                        "partial RoPE")
+                        "partial RoPE; 8: workload 4 with FP8 cache entries")
     return p.parse_args()
 
 
@@ -430,6 +430,26 @@ def other_workload_plan(wid, wl, csa, torch, D):
                                                       "partial RoPE: indexer + top-k, attention with the "
                                                       "query's norm / rotation and the output's inverse "
                                                       "rotation fused in")
+    if wid == 8:
+        B, nc, H, d, dI, HI = s["B"], s["nc"], s["H"], s["d"], s["dI"], s["HI"]
+        # the entry cache as the decode step keeps it: FP8 codes, scales, bf16 RoPE dims
+        D["kv_fp8"], D["kv_sc"], D["kv_rope"] = csa.csa_quantize_fp8_entries(D["kv"])
+        D["kv_sc"] = D["kv_sc"].view(B, nc)
+        torch.cuda.synchronize()
+        idx = torch.empty(B, 1, k, dtype=torch.int32, device="cuda")
+        out = torch.empty(B, 1, H, d, dtype=torch.bfloat16, device="cuda")
+        ws = csa.index_topk_workspace(B, 1, nc, False)
+        stages = [
+            ("csa_index_topk", lambda: csa.csa_index_topk(D["qI"], D["w"], D["kI"], D["lens"], k,
+                                                          idx_out=idx, workspace=ws)),
+            ("csa_attend_fp8", lambda: csa.csa_attend_fp8(D["q"], D["kv_fp8"], D["kv_sc"], D["kv_rope"], D["win"],
+                                                          idx, D["lens"], window=window, out=out)),
+        ]
+        byts = B * (nc * dI * 2 + k * (64 + 1 + 128) + window * d * 2 + (2 * H * d + HI * dI + HI) * 2)
+        flops = B * (2.0 * nc * HI * dI + 4.0 * (k + window) * H * d)
+        return stages, "queries/s", B, byts, flops, ("one decode step of the 1M workload with FP8 cache entries "
+                                                      "(64 E4M3 dims + scale + 64 bf16 RoPE dims): indexer + "
+                                                      "top-k, attention widening the selected entries on chip")
     if wid == 5:
         B, H, d, dI, HI, m = s["B"], s["H"], s["d"], s["dI"], s["HI"], s["m"]
         nc = s["nc"]
@@ -464,7 +484,7 @@ def run_other_workload(args):
     from tests.helpers import to_dev
     torch.cuda.set_device(0)
     wid = args.workload
-    wl = W.make(4 if wid in (6, 7) else wid)
+    wl = W.make(4 if wid in (6, 7, 8) else wid)
     D = {n: to_dev(wl[n]) for n in wl.arrays if n != "needle_pos"}
     stages, unit, units, byts, flops, what = other_workload_plan(wid, wl, csa, torch, D)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
@@ -518,7 +538,8 @@ def run_other_workload(args):
     tfl = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     gbs = byts / (ms * 1e-3) / 1e9
     tfs = flops / (ms * 1e-3) / 1e12
-    name = {6: "csa_decode_mxfp4keys_b4_n1048576", 7: "csa_decode_qknorm_rope_b4_n1048576"}.get(wid, wl.name)
+    name = {6: "csa_decode_mxfp4keys_b4_n1048576", 7: "csa_decode_qknorm_rope_b4_n1048576",
+            8: "csa_decode_fp8entries_b4_n1048576"}.get(wid, wl.name)
     line = {"metric": f"{name}: {unit}", "value": units * 1000.0 / ms, "unit": unit, "n_gpus": 1,
             "steps": K, "warmup": max(3, args.warmup), "ms_per_step": ms, "higher_is_better": True,
             "dtype": wl.dt, "data": "synthetic (seeded PCG64)",
@@ -536,6 +557,8 @@ def run_other_workload(args):
         line["compress_step"] = time_compress_step(wl, csa, torch, D, flush, min(K, 20))
     if wid == 7:
         line["norm_rope_cache"] = time_norm_rope_cache(wl, csa, torch, D, min(K, 50), hbm)
+    if wid == 8:
+        line["quantize_fp8_cache"] = time_quantize_fp8_cache(wl, csa, torch, D, min(K, 50), hbm)
     if not args.no_cpu_baseline:
         line["cpu_baseline"] = oracle_sample(wid, wl)
     print(json.dumps(line))
@@ -589,6 +612,18 @@ def oracle_sample(wid, wl):
         t = clock(one)
         return {"value": 1.0 / t, "unit": "queries/s", "cores": cores, "kind": "oracle",
                 "sample": "one query of the batch (its keys quantised, dequantised, scored; attention)"}
+    if wid == 8:
+        sl = slice(0, 1)
+        # the cache as the step finds it (quantised when the entries are formed)
+        f8, sc8, rp8 = oracle.quantize_fp8_entries(wl["kv"][sl])
+        deq = oracle.round_to(oracle.dequant_fp8_entries(f8, sc8, rp8), oracle.BF16)
+
+        def one():
+            idx, _ = oracle.index_topk(wl["qI"][sl], wl["w"][sl], wl["kI"][sl], wl["lens"][sl], k)
+            oracle.attend(wl["q"][sl], deq, wl["win"][sl], wl["lens"][sl], idx=idx, window=window)
+        t = clock(one)
+        return {"value": 1.0 / t, "unit": "queries/s", "cores": cores, "kind": "oracle",
+                "sample": "one query of the batch (indexer + top-k, attention over the dequantised FP8 entries)"}
     if wid == 7:
         sl = slice(0, 1)
         d, nc = s["d"], s["nc"]
@@ -710,6 +745,28 @@ def time_norm_rope_cache(wl, csa, torch, D, K, hbm):
     byts = 2 * B * nc * d * 2
     gbs = byts / (us * 1e-6) / 1e9
     return {"kernel": "k_norm_rope<bf16,128>", "rows": B * nc, "us": us, "bytes_per_launch": byts,
+            "achieved_gbs": gbs, "frac_of_measured_hbm": gbs / hbm, "bound": "hbm"}
+
+
+def time_quantize_fp8_cache(wl, csa, torch, D, K, hbm):
+    """csa_quantize_fp8_entries over the whole 1M-token entry cache (B x
+    262,144 entries: 256 B read, 64 + 1 + 128 B written per entry)."""
+    s = wl.sizes
+    B, nc, d = s["B"], s["nc"], s["d"]
+    for _ in range(3):
+        csa.csa_quantize_fp8_entries(D["kv"])
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    for a, b in ev:
+        a.record()
+        csa.csa_quantize_fp8_entries(D["kv"])
+        b.record()
+    torch.cuda.synchronize()
+    csa.check_device_error()
+    us = 1000 * statistics.median(a.elapsed_time(b) for a, b in ev)
+    byts = B * nc * (d * 2 + 64 + 1 + 128)
+    gbs = byts / (us * 1e-6) / 1e9
+    return {"kernel": "k_quantize_fp8_entries<bf16>", "rows": B * nc, "us": us, "bytes_per_launch": byts,
             "achieved_gbs": gbs, "frac_of_measured_hbm": gbs / hbm, "bound": "hbm"}
 
 
