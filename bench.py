@@ -457,13 +457,17 @@ def other_workload_plan(wid, wl, csa, torch, D):
         out_c = torch.empty(B, 1, H, d, dtype=torch.bfloat16, device="cuda")
         out_h = torch.empty(B, 1, H, d, dtype=torch.bfloat16, device="cuda")
         ws = csa.index_topk_workspace(B, 1, nc, False)
+        # the layer-pair scheduler: one call, the HCA attention beside the CSA layer
         stages = [
-            ("csa_index_topk", lambda: csa.csa_index_topk(D["qI"], D["w"], D["kI"], D["lens"], k,
-                                                          idx_out=idx, workspace=ws)),
-            ("csa_attend", lambda: csa.csa_attend(D["q"], D["kv"], D["win"], idx, D["lens"],
-                                                  window=window, out=out_c)),
-            ("hca_attend", lambda: csa.hca_attend(D["q2"], D["hkv"], D["win"], D["lens"], m=m,
-                                                  window=window, out=out_h)),
+            ("csa_hca_pair_decode", lambda: csa.csa_hca_pair_decode(
+                D["q"], D["qI"], D["w"], D["kI"], D["kv"], D["q2"], D["hkv"], D["win"], D["lens"], k, m=m,
+                window=window, idx_out=idx, out_csa=out_c, out_hca=out_h, workspace=ws)),
+        ]
+        # the same step as three calls on one stream, timed beside it
+        D["serial_step"] = [
+            lambda: csa.csa_index_topk(D["qI"], D["w"], D["kI"], D["lens"], k, idx_out=idx, workspace=ws),
+            lambda: csa.csa_attend(D["q"], D["kv"], D["win"], idx, D["lens"], window=window, out=out_c),
+            lambda: csa.hca_attend(D["q2"], D["hkv"], D["win"], D["lens"], m=m, window=window, out=out_h),
         ]
         lens = wl["lens"].astype(np.int64)
         vis, hv = lens // 4, lens // m
@@ -555,6 +559,10 @@ def run_other_workload(args):
         line["hca_compress"] = time_hca_compress(wl, csa, torch, flush, min(K, 20), hbm)
     if wid == 5:
         line["compress_step"] = time_compress_step(wl, csa, torch, D, flush, min(K, 20))
+        ser = time_step_graph(D["serial_step"], K, flush, torch, csa)
+        line["serial_three_calls"] = {"ms_per_step": ser, "value": units * 1000.0 / ser,
+                                      "note": "csa_index_topk, csa_attend, hca_attend on one stream, "
+                                              "timed the same way"}
     if wid == 7:
         line["norm_rope_cache"] = time_norm_rope_cache(wl, csa, torch, D, min(K, 50), hbm)
     if wid == 8:
@@ -670,6 +678,36 @@ def oracle_sample(wid, wl):
         return {"value": nq / t, "unit": "queries/s", "cores": cores, "kind": "oracle",
                 "sample": f"the CSA + HCA step for {nq} of the {s['B']} sequences"}
     raise KeyError(wid)
+
+
+def time_step_graph(fns, K, flush, torch, csa):
+    """Median device time (ms) of the calls `fns` replayed from a CUDA graph,
+    the L2 flushed before every step (as the workload lines are timed)."""
+    def step():
+        for fn in fns:
+            fn()
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize()
+    run = step
+    try:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            step()
+        g.replay()
+        torch.cuda.synchronize()
+        run = g.replay
+    except Exception:
+        torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    for a, b in ev:
+        flush.zero_()
+        a.record()
+        run()
+        b.record()
+    torch.cuda.synchronize()
+    csa.check_device_error()
+    return statistics.median(a.elapsed_time(b) for a, b in ev)
 
 
 def time_compress_step(wl, csa, torch, D, flush, K):

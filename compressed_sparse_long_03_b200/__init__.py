@@ -73,6 +73,8 @@ def lib() -> ctypes.CDLL:
         L.hca_attend.argtypes = [P, P, P, I, P, P, I, I, I, I, I, I, I, F, P, I, P, P]
         L.csa_norm_rope.argtypes = [P, P, ctypes.c_long, I, I, P, P, I, I, I, P, F, I, F, I, I, P]
         L.csa_quantize_fp8_entries.argtypes = [P, ctypes.c_long, I, I, I, P, P, P, P]
+        L.csa_hca_pair_decode.argtypes = [P, P, P, P, P, I, I, I, I, P, P, I, I, P, I, P, I, I, I, I, P, P, P,
+                                          P, S, P]
         L.csa_attend_fp8.argtypes = [P, P, P, P, P, I, P, P, P, I, I, I, I, I, I, I, F, P, I, P, P]
         L.hca_attend_fp8.argtypes = [P, P, P, P, P, I, P, P, I, I, I, I, I, I, I, F, P, I, P, P]
         L.csa_attend_rope.argtypes = [P, P, P, I, P, P, P, I, I, I, I, I, I, I, F, P, P, F, I, F, I, I, P, P]
@@ -422,3 +424,26 @@ def hca_attend_fp8(q, kv_fp8, kv_scales, kv_rope, kv_tok, lens, q_pos=None, m=12
                                 _i32(lens), _i32(q_pos), B, Tq, H, d, kv_fp8.shape[1], m, window, float(scale),
                                 _f32(sink), _dt(q), _p(out), _s(stream)))
     return out
+
+
+def csa_hca_pair_decode(q_csa, q_idx, w, k_idx, kv_csa, q_hca, kv_hca, kv_tok, lens, k, m=128, window=128,
+                        idx_out=None, out_csa=None, out_hca=None, workspace=None, stream=None):
+    """One decode step of a CSA + HCA layer pair in one call (the HCA
+    attention beside the CSA layer on a second stream) -> (idx_out, out_csa,
+    out_hca)."""
+    B, _, H, d = q_csa.shape
+    HI, dI = q_idx.shape[-2], q_idx.shape[-1]
+    nc_max, nh_max = k_idx.shape[1], kv_hca.shape[1]
+    if idx_out is None:
+        idx_out = torch.empty(B, 1, k, dtype=torch.int32, device=q_csa.device)
+    if out_csa is None:
+        out_csa = torch.empty_like(q_csa)
+    if out_hca is None:
+        out_hca = torch.empty_like(q_hca)
+    if workspace is None:
+        workspace = index_topk_workspace(B, 1, nc_max, False)
+    _check(lib().csa_hca_pair_decode(_p(q_csa), _p(q_idx), _p(w), _p(k_idx), _p(kv_csa), nc_max, HI, dI, int(k),
+                                     _p(q_hca), _p(kv_hca), nh_max, int(m), _p(kv_tok), kv_tok.shape[1],
+                                     _i32(lens), B, H, d, int(window), _i32(idx_out), _p(out_csa), _p(out_hca),
+                                     _p(workspace), workspace.numel() * workspace.element_size(), _s(stream)))
+    return idx_out, out_csa, out_hca

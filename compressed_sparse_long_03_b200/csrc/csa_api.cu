@@ -58,6 +58,9 @@ struct TimingSlot {
   int dev = -1;
 };
 thread_local bool g_timing = false;
+// CTAs of the persistent scoring kernel (0: one per SM); the layer-pair
+// step lowers it to leave SMs to the HCA attention running beside it
+thread_local int g_score_ctas = 0;
 thread_local std::vector<TimingSlot> g_slots;
 thread_local int g_nlaunch = 0;
 
@@ -415,7 +418,8 @@ int launch_index_tc(const void *qI, const void *w, const void *kI, const int32_t
   a.U = B * a.gpb;
   a.stages = stages;
   a.fill_invisible = fill ? 1 : 0;
-  return launch_cluster(kern, 1, (unsigned)num_sms(), csa::kTcThreads, smem, st, what, tmK, tmQ, a);
+  const int ctas = g_score_ctas > 0 ? std::min(g_score_ctas, num_sms()) : num_sms();
+  return launch_cluster(kern, 1, (unsigned)ctas, csa::kTcThreads, smem, st, what, tmK, tmQ, a);
 }
 
 // Decode (one query row per sequence): one row per unit, the heads padded to
@@ -962,6 +966,105 @@ int hca_attend(const void *q, const void *kv_c, const void *kv_tok, int n_tok,
   if (nc_max > 65536) return fail(CSA_ERR_UNSUPPORTED, "hca_attend: nc_max=%d > 65536", nc_max);
   return attend_common(q, kv_c, kv_tok, n_tok, nullptr, lens, q_pos, B, Tq, H, d, nc_max, 0, m,
                        window, scale, sink, dt, out, stream, "hca_attend");
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// The CSA + HCA layer pair of one decode step as one call (the scheduler).
+// "Anatomy of a Frontier Model", "The attention: compress, then select": V4
+// interleaves CSA and HCA layers.  With both layers' queries given, the HCA
+// attention shares nothing with the CSA layer's scoring, selection and
+// attention, so it runs on a second stream beside them: the persistent
+// scoring kernel is launched on all but a quarter of the SMs (at most one
+// per HCA row), and the HCA attention fills the rest from a high-priority
+// stream, ahead of the selection's early-launched CTAs.  Fork and join are
+// event edges, so the call can be captured into a CUDA graph with both
+// branches.
+// ---------------------------------------------------------------------------
+namespace {
+
+struct PairCtx {
+  cudaStream_t side = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+};
+std::mutex g_pair_mu;
+PairCtx g_pair[64];
+
+int pair_ctx(PairCtx **out, const char *what) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess || dev < 0 || dev >= 64) return fail(CSA_ERR_CUDA, "%s: no usable device", what);
+  std::lock_guard<std::mutex> lock(g_pair_mu);
+  PairCtx &c = g_pair[dev];
+  if (!c.side) {
+    int least = 0, greatest = 0;
+    e = cudaDeviceGetStreamPriorityRange(&least, &greatest);
+    if (e == cudaSuccess) e = cudaStreamCreateWithPriority(&c.side, cudaStreamNonBlocking, greatest);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&c.fork, cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&c.join, cudaEventDisableTiming);
+    if (e != cudaSuccess) {
+      c = PairCtx();
+      return fail(CSA_ERR_CUDA, "%s: creating the pair stream: %s", what, cudaGetErrorString(e));
+    }
+  }
+  *out = &c;
+  return CSA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int csa_hca_pair_decode(const void *q_csa, const void *q_idx, const void *w, const void *k_idx, const void *kv_csa,
+                        int nc_max, int HI, int dI, int k, const void *q_hca, const void *kv_hca, int nh_max, int m,
+                        const void *kv_tok, int n_tok, const int32_t *lens, int B, int H, int d, int window,
+                        int32_t *idx_out, void *out_csa, void *out_hca, void *workspace, size_t ws_bytes,
+                        void *stream) {
+  const char *what = "csa_hca_pair_decode";
+  begin_call();
+  const csa_dtype dt = CSA_BF16;
+  int rc = check_index_args(what, dt, B, 1, HI, dI, nc_max);
+  if (rc) return rc;
+  rc = check_topk_args(what, B, 1, nc_max, k);
+  if (rc) return rc;
+  if (m < 1 || m > 4096) return fail(CSA_ERR_UNSUPPORTED, "%s: m=%d not in [1,4096]", what, m);
+  if (nh_max < 0 || nh_max > 65536) return fail(CSA_ERR_UNSUPPORTED, "%s: nh_max=%d not in [0,65536]", what, nh_max);
+  if (B == 0) return CSA_OK;
+  if (!q_csa || !q_idx || !w || !lens || !idx_out || !out_csa || !out_hca || !q_hca || !kv_tok ||
+      (nc_max > 0 && (!k_idx || !kv_csa)) || (nh_max > 0 && !kv_hca))
+    return fail(CSA_ERR_NULL, "%s: a required pointer is NULL", what);
+  if (!aligned16(q_idx) || !aligned16(w) || (k_idx && !aligned16(k_idx)))
+    return fail(CSA_ERR_ALIGN, "%s: tensors must be 16-byte aligned", what);
+  const size_t need = csa_index_topk_workspace_size(B, 1, nc_max, 0);
+  if (need > 0 && (!workspace || ws_bytes < need || !aligned16(workspace)))
+    return fail(CSA_ERR_WORKSPACE, "%s: a 16-byte aligned workspace of %zu B is needed", what, need);
+  PairCtx *pc = nullptr;
+  rc = pair_ctx(&pc, what);
+  if (rc) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  float *scores = static_cast<float *>(workspace);
+  // fork before the first CSA kernel: the HCA branch may start at once
+  cudaError_t e = cudaEventRecord(pc->fork, st);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(pc->side, pc->fork, 0);
+  if (e != cudaSuccess) return fail(CSA_ERR_CUDA, "%s: fork: %s", what, cudaGetErrorString(e));
+  const int sms = num_sms();
+  g_score_ctas = sms - std::max(1, std::min(B, sms / 4));
+  rc = index_scores_impl(q_idx, w, k_idx, lens, nullptr, B, 1, HI, dI, nc_max, dt, scores, false, st);
+  g_score_ctas = 0;
+  if (!rc)
+    rc = attend_common(q_hca, kv_hca, kv_tok, n_tok, nullptr, lens, nullptr, B, 1, H, d, nh_max, 0, m, window,
+                       0.f, nullptr, dt, out_hca, pc->side, what);
+  if (!rc) rc = topk_impl(scores, lens, nullptr, B, 1, nc_max, k, idx_out, st);
+  if (!rc)
+    rc = attend_common(q_csa, kv_csa, kv_tok, n_tok, idx_out, lens, nullptr, B, 1, H, d, nc_max, k, 4, window,
+                       0.f, nullptr, dt, out_csa, st, what);
+  // join, whatever happened above: the caller's stream (or capture) stays whole
+  e = cudaEventRecord(pc->join, pc->side);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(st, pc->join, 0);
+  if (rc) return rc;
+  if (e != cudaSuccess) return fail(CSA_ERR_CUDA, "%s: join: %s", what, cudaGetErrorString(e));
+  return CSA_OK;
 }
 
 int csa_quantize_fp8_entries(const void *kv, long rows, int d, int rope_dim, csa_dtype dt, uint8_t *fp8,

@@ -426,6 +426,36 @@ CSA_API int hca_attend_fp8(const void *q, const uint8_t *kv_fp8, const uint8_t *
                            int H, int d, int nc_max, int m, int window, float scale, const float *sink,
                            csa_dtype dt, void *out, void *stream);
 
+/* ------------------------------------------------------------------------
+ * csa_hca_pair_decode -- one decode step of an interleaved CSA + HCA layer
+ * pair (Anatomy page, "The attention: compress, then select": V4
+ * interleaves the two kinds of layer), both layers' queries given, issued as
+ * one call:
+ *   idx_out = csa_index_topk(q_idx, w, k_idx, ...)          (CSA, m = 4)
+ *   out_csa = csa_attend(q_csa, kv_csa, kv_tok, idx_out, ...)
+ *   out_hca = hca_attend(q_hca, kv_hca, kv_tok, ..., m)     (HCA)
+ * with one query row per sequence (Tq = 1, decode positions lens[b] - 1),
+ * bf16, default softmax scale, no sink.  The results are those of the three
+ * calls.  Scheduling: the HCA attention shares nothing with the CSA layer,
+ * so it runs on a second (library-owned, high-priority) stream forked from
+ * and joined back to `stream` by events; the persistent CSA scoring kernel
+ * is launched on all but min(B, SMs / 4) SMs so that the HCA rows run beside
+ * it.  Capturable into a CUDA graph (fork and join are event edges).
+ *   q_csa, q_hca [B][1][H][d]; q_idx [B][1][HI][dI]; w [B][1][HI];
+ *   k_idx [B][nc_max][dI]; kv_csa [B][nc_max][d]; kv_hca [B][nh_max][d];
+ *   kv_tok [B][n_tok][d] (the window ring both layers read);
+ *   idx_out [B][1][k]; out_csa, out_hca [B][1][H][d];
+ *   workspace >= csa_index_topk_workspace_size(B, 1, nc_max, 0) bytes.
+ * Supported sets: those of the three calls.  The library creates its
+ * second stream and two events once per device, on the first call (before
+ * any capture).
+ * ---------------------------------------------------------------------- */
+CSA_API int csa_hca_pair_decode(const void *q_csa, const void *q_idx, const void *w, const void *k_idx,
+                                const void *kv_csa, int nc_max, int HI, int dI, int k, const void *q_hca,
+                                const void *kv_hca, int nh_max, int m, const void *kv_tok, int n_tok,
+                                const int32_t *lens, int B, int H, int d, int window, int32_t *idx_out,
+                                void *out_csa, void *out_hca, void *workspace, size_t ws_bytes, void *stream);
+
 #ifdef __cplusplus
 }
 #endif
