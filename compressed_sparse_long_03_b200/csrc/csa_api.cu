@@ -1083,6 +1083,19 @@ int csa_quantize_fp8_entries(const void *kv, long rows, int d, int rope_dim, csa
   if (!aligned16(kv) || (fp8 && (reinterpret_cast<uintptr_t>(fp8) & 1)) || (rope && !aligned16(rope)))
     return fail(CSA_ERR_ALIGN, "%s: kv and rope 16-byte aligned, fp8 2-byte aligned", what);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // eight elements per lane when a row is 8, 16 or 32 lanes and the planes
+  // take 8- and 16-byte vectors
+  const bool v8 = (d == 64 || d == 128 || d == 256) && !(reinterpret_cast<uintptr_t>(fp8) & 7);
+  if (v8) {
+    const long per_cta = 8L * (32 / (d / 8));
+    const unsigned g8 = (unsigned)std::max(1L, std::min((rows + per_cta - 1) / per_cta, 8L * num_sms()));
+    if (dt == CSA_F32)
+      return launch_cluster(csa::k_quantize_fp8_entries_v8<float>, 1, g8, csa::kF8Threads, 0, st, what,
+                            static_cast<const float *>(kv), rows, d, rope_dim, fp8, scales, static_cast<float *>(rope));
+    return launch_cluster(csa::k_quantize_fp8_entries_v8<__nv_bfloat16>, 1, g8, csa::kF8Threads, 0, st, what,
+                          static_cast<const __nv_bfloat16 *>(kv), rows, d, rope_dim, fp8, scales,
+                          static_cast<__nv_bfloat16 *>(rope));
+  }
   const unsigned grid = (unsigned)std::max(1L, std::min((rows + 7) / 8, 8L * num_sms()));
   if (dt == CSA_F32)
     return launch_cluster(csa::k_quantize_fp8_entries<float>, 1, grid, csa::kF8Threads, 0, st, what,

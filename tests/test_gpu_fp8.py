@@ -35,7 +35,7 @@ def _edge_rows(d, dt):
 
 
 @pytest.mark.parametrize("dt", ["bf16", "f32"])
-@pytest.mark.parametrize("d,r", [(128, 64), (256, 64), (64, 0)])
+@pytest.mark.parametrize("d,r", [(128, 64), (256, 64), (64, 0), (192, 64)])
 def test_quantize_fp8_bit_exact(dt, d, r):
     x = W.normal(40 + d + r, "kv", (1000, d), 2.0, dt)
     x = np.concatenate([x, _edge_rows(d, dt)])
