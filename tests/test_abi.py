@@ -182,3 +182,20 @@ def test_fp8_entries_validation(L):
     assert att(codes=None) == E_NULL
     assert att(rope=A4) == E_ALIGN
     assert att("hca_attend_fp8", nc=65540) == E_UNSUP
+
+
+def test_pair_decode_validation(L):
+    def pair(**kw):
+        a = dict(nc=8, HI=4, dI=128, k=4, nh=4, m=128, B=1, H=4, d=128, ws=A16, ws_bytes=1 << 20, q=A16)
+        a.update(kw)
+        return L.csa_hca_pair_decode(a["q"], A16, A16, A16, A16, a["nc"], a["HI"], a["dI"], a["k"], A16, A16,
+                                     a["nh"], a["m"], A16, 128, A16, a["B"], a["H"], a["d"], 128, A16, A16, A16,
+                                     a["ws"], a["ws_bytes"], None)
+    assert pair(m=0) == E_UNSUP
+    assert pair(nh=70000) == E_UNSUP
+    assert pair(dI=96) == E_UNSUP
+    assert pair(HI=0) == E_UNSUP
+    assert pair(q=None) == E_NULL
+    assert pair(ws=None) == E_WS
+    assert pair(ws_bytes=16) == E_WS
+    assert pair(B=0) == OK
