@@ -47,6 +47,7 @@ struct AttendArgs {
   void *out;
   const float *sink;  // [H] per-head sink logits (scaled-logit units), or nullptr
   int n_tok, k, Tq, H, nc_max, m, window;
+  int R;             // query rows B * Tq
   float scale_log2;  // softmax scale * log2(e)
   // QK-norm and partial RoPE fused around the attention (third of the three
   // details): qk_flags kNrNorm normalises each query head (q_gamma [d] or

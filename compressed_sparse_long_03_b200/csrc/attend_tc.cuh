@@ -88,14 +88,11 @@ __global__ void __launch_bounds__(kAtThreads, 1) k_attend_tc(AttendArgs a) {
   const __nv_bfloat16 *kv_rp = static_cast<const __nv_bfloat16 *>(a.kv_rope);
 
   const int rank = (CS > 1) ? (int)cg::this_cluster().block_rank() : 0;
-  const int r = blockIdx.x / CS;
-  const int b = r / a.Tq, tq = r % a.Tq;
   const int tid = threadIdx.x, warp = tid >> 5;
   const int H = a.H;
   const __nv_bfloat16 *q = static_cast<const __nv_bfloat16 *>(a.q);
   const __nv_bfloat16 *kv_c = static_cast<const __nv_bfloat16 *>(a.kv_c);
   const __nv_bfloat16 *kv_tok = static_cast<const __nv_bfloat16 *>(a.kv_tok);
-  __nv_bfloat16 *out = static_cast<__nv_bfloat16 *>(a.out) + (size_t)r * H * D;
 
   // set-up that touches no global memory runs before the wait on the
   // previous kernel: barriers and the TMEM allocation
@@ -111,6 +108,13 @@ __global__ void __launch_bounds__(kAtThreads, 1) k_attend_tc(AttendArgs a) {
   }
   pdl_wait();
   pdl_launch_dependents();
+  uint32_t ns = 0, no = 0;  // mbarrier phases, carried from row to row
+  bool cta_alive = true;
+  // one query row per cluster; with one CTA per row (CS == 1) the CTAs are
+  // persistent and take rows blockIdx.x, blockIdx.x + gridDim.x, ...
+  for (int r = blockIdx.x / CS; r < a.R && cta_alive; r += (CS == 1 ? (int)gridDim.x : a.R)) {
+  const int b = r / a.Tq, tq = r % a.Tq;
+  __nv_bfloat16 *out = static_cast<__nv_bfloat16 *>(a.out) + (size_t)r * H * D;
   // Q rows (heads) in the swizzled K-major layout; heads >= H are zero rows
   const __nv_bfloat16 *qrow = q + (size_t)r * H * D;
   for (int u = tid; u < 128 * 16; u += kAtThreads) {
@@ -140,13 +144,8 @@ __global__ void __launch_bounds__(kAtThreads, 1) k_attend_tc(AttendArgs a) {
     for (int u = tid; u < H * D; u += kAtThreads)
       if ((u / D) % CS == rank) out[u] = __float2bfloat16_rn(0.f);
     cp_async_wait_all();
-    tc_fence_before();
-    __syncthreads();
-    if (warp == 0) {
-      tc_fence_after();
-      tmem_dealloc(tmem_holder, 512);
-    }
-    return;
+    __syncthreads();  // Q's buffer is free for the next row
+    continue;
   }
 
   const int nsel = a.idx ? a.k : v;
@@ -172,7 +171,6 @@ __global__ void __launch_bounds__(kAtThreads, 1) k_attend_tc(AttendArgs a) {
 #pragma unroll
   for (int e = 0; e < D / 2; ++e) o[e] = 0.f;
   float m_run = -INFINITY, l_run = 0.f;  // l_run: this half's share of the sum
-  uint32_t ns = 0, no = 0;
   bool alive = true;
 
   // row pointers (one coalesced index read) and validity words of the tile
@@ -545,6 +543,11 @@ __global__ void __launch_bounds__(kAtThreads, 1) k_attend_tc(AttendArgs a) {
     *reinterpret_cast<uint2 *>(out + (size_t)h * D + 4 * j) = pk;
   }
   }  // clusters
+  if (!alive) cta_alive = false;  // a wait gave up: no further rows
+  tc_fence_before();
+  __syncthreads();  // every thread is done with this row's Q, tiles, P and TMEM reads
+  tc_fence_after();
+  }  // rows
   if (tid == 0 && abort_flag) raise_dev_err(kDevErrTimeout);
   tc_fence_before();
   __syncthreads();

@@ -584,7 +584,10 @@ int launch_attend_tc(const csa::AttendArgs &a, int R, cudaStream_t st, const cha
   const size_t smem = csa::at_smem_bytes(cs, a.kv_fp8 != nullptr);
   int rc = ensure_smem(kern, smem, what);
   if (rc) return rc;
-  return launch_cluster(kern, cs, (unsigned)cs * R, csa::kAtThreads, smem, st, what, a);
+  // clusters: one per row; one CTA per row: persistent CTAs, one per SM,
+  // each looping over rows (set-up and TMEM allocation once per SM)
+  const unsigned grid = cs == 1 ? (unsigned)std::min(R, num_sms()) : (unsigned)cs * R;
+  return launch_cluster(kern, cs, grid, csa::kAtThreads, smem, st, what, a);
 }
 
 // QK-norm / partial RoPE arguments of the fused attention entry points.
@@ -674,6 +677,7 @@ int attend_common(const void *q, const void *kv_c, const void *kv_tok, int n_tok
   a.nc_max = nc_max;
   a.m = m;
   a.window = window;
+  a.R = B * Tq;
   const float sc = scale > 0.f ? scale : 1.0f / sqrtf((float)d);
   a.scale_log2 = sc * 1.4426950408889634f;
   a.qk_flags = qk.flags;
