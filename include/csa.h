@@ -38,6 +38,21 @@
  *    complete): a query at position t sees compressed entries
  *    i < floor((t+1)/m) (m = 4 for CSA), plus the window tokens
  *    max(0, t-window+1) .. t.
+ *  - The one host-side resource the library creates is the second stream
+ *    and two events of csa_hca_pair_decode, once per device.
+ *
+ * Entry points, in the order below
+ *  - compression: csa_compress, hca_compress; at decode, one entry per
+ *    completed block: csa_compress_step, hca_compress_step;
+ *  - selection: csa_index_topk (= csa_index_scores + csa_topk), the
+ *    allocation-free csa_index_topk_noalloc, and over MXFP4 indexer keys
+ *    csa_quantize_mxfp4 + csa_index_topk_mxfp4;
+ *  - attention: csa_attend, hca_attend (optional sink); with QK-norm and
+ *    partial RoPE fused, csa_attend_rope, hca_attend_rope, and the cache
+ *    pass csa_norm_rope; over FP8 entries, csa_quantize_fp8_entries +
+ *    csa_attend_fp8, hca_attend_fp8;
+ *  - scheduling: csa_hca_pair_decode, one decode step of a CSA + HCA layer
+ *    pair as one call.
  */
 #ifndef CSA_B200_H
 #define CSA_B200_H
