@@ -41,7 +41,7 @@
  *  - The one host-side resource the library creates is the second stream
  *    and two events of csa_hca_pair_decode, once per device.
  *
- * Entry points, in the order below
+ * Entry points, by role
  *  - compression: csa_compress, hca_compress; at decode, one entry per
  *    completed block: csa_compress_step, hca_compress_step;
  *  - selection: csa_index_topk (= csa_index_scores + csa_topk), the
